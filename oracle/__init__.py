@@ -1,0 +1,188 @@
+"""Float64 CPU oracle for decoupled-head attention. TEST INFRASTRUCTURE ONLY.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the ``cpu_baseline`` /
+``--impl reference`` legs of ``bench.py`` may import this package. The CUDA
+library never does, and this package imports nothing from it.
+
+What it computes is the plain definition, written out step by step:
+
+* Head -> group map. Query head i reads key/value group g(i) = floor(i*H_kv/H_q).
+  For H_q divisible by H_kv this is i // (H_q/H_kv): contiguous blocks of query
+  heads share one group, as drawn in the GQA explainer ("GQA -- Grouped-Query
+  Attention", head-to-group diagram: Q1..Q4 -> KV1, Q5..Q8 -> KV2), and as its
+  PyTorch module builds it with ``unsqueeze(2).expand(...)`` ("PyTorchでのGQA実装").
+  G = H gives MHA, G = 1 gives MQA (same page, "MHA・MQA・GQAの関係").
+  Sparse Query Attention changes only H_q ("Sparse Query Attention (SQA)", abstract).
+* Explicit repetition. For each query head the group's K and V are copied out
+  into that head's own matrices before any arithmetic.
+* Scores. s_u = scale * <q_t, k_u> over keys u (all keys, or u <= t when causal:
+  ``scaled_dot_product_attention(..., is_causal=True)`` in the GQA module);
+  masked keys are excluded (exp(-inf) = 0 exactly).
+* Two-pass softmax. m = max_u s_u; e_u = exp(s_u - m); l = sum_u e_u;
+  out = (sum_u e_u v_u) / l.
+* Layer. q/k/v = x W^T with no bias, viewed [B, N, H, d]; attention as above;
+  heads merged back to [B, N, H_q*d]; out = A Wo^T (the GQA module's
+  ``q_proj/k_proj/v_proj/o_proj`` with ``bias=False``).
+
+Everything is float64 from the exact bf16 values. Library matmuls (numpy/BLAS)
+serve as the dot-product step; nothing else is blocked, fused or reordered.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+__all__ = [
+    "group_of_head", "repeat_kv", "widen_bf16", "bf16_round", "attention",
+    "attention_rows", "linear", "layer", "layer_rows",
+]
+
+
+def group_of_head(i: int, H_q: int, H_kv: int) -> int:
+    """KV group read by query head i: floor(i * H_kv / H_q)."""
+    return (i * H_kv) // H_q
+
+
+def widen_bf16(bits) -> np.ndarray:
+    """bf16 bit patterns (uint16) -> float64, exactly."""
+    b = np.ascontiguousarray(bits, dtype=np.uint16)
+    return (b.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def bf16_round(a: np.ndarray) -> np.ndarray:
+    """Round float64 values to the nearest bfloat16 (ties to even), returned as float64.
+
+    bfloat16 keeps 7 fraction bits; from a float64 that drops the low 45 of 52.
+    Only the normal bf16 range is needed here (inputs are O(1)); values below
+    2^-126 in magnitude are rounded on the float32 grid first, which is exact
+    for them.
+    """
+    a = np.asarray(a, dtype=np.float64)
+    bits = a.view(np.uint64).copy()
+    sign = bits & np.uint64(0x8000000000000000)
+    mag = bits & np.uint64(0x7FFFFFFFFFFFFFFF)
+    lsb = (mag >> np.uint64(45)) & np.uint64(1)
+    mag = (mag + np.uint64((1 << 44) - 1) + lsb) & ~np.uint64((1 << 45) - 1)
+    out = (sign | mag).view(np.float64)
+    tiny = np.abs(a) < 2.0 ** -126
+    if np.any(tiny):
+        f = a[tiny].astype(np.float32).view(np.uint32).astype(np.uint64)
+        flsb = (f >> np.uint64(16)) & np.uint64(1)
+        f = (f + np.uint64(0x7FFF) + flsb) & np.uint64(0xFFFF0000)
+        out[tiny] = f.astype(np.uint32).view(np.float32).astype(np.float64)
+    return out
+
+
+def repeat_kv(kv: np.ndarray, H_q: int) -> np.ndarray:
+    """[B, N, H_kv, d] -> [B, N, H_q, d], head i holding a copy of group g(i)."""
+    B, N, H_kv, d = kv.shape
+    out = np.empty((B, N, H_q, d), dtype=np.float64)
+    for i in range(H_q):
+        out[:, :, i, :] = kv[:, :, group_of_head(i, H_q, H_kv), :]
+    return out
+
+
+def _softmax_rows_times_v(s: np.ndarray, vh: np.ndarray) -> np.ndarray:
+    """Two-pass softmax of each score row, then the weighted sum of values."""
+    m = np.max(s, axis=1, keepdims=True)          # pass 1: row max
+    e = np.exp(s - m)                              # pass 2: exponentials (masked -> 0)
+    l = np.sum(e, axis=1, keepdims=True)
+    return (e @ vh) / l
+
+
+def _head_rows(qh, kh, vh, t_idx, causal, scale, chunk):
+    """Attention of query rows ``qh`` (tokens ``t_idx``) of one head against kh, vh."""
+    N = kh.shape[0]
+    out = np.empty((qh.shape[0], vh.shape[1]), dtype=np.float64)
+    keys = np.arange(N)
+    for a in range(0, qh.shape[0], chunk):
+        b = min(a + chunk, qh.shape[0])
+        s = scale * (qh[a:b] @ kh.T)              # explicit score rows
+        if causal:
+            s[keys[None, :] > t_idx[a:b, None]] = -np.inf
+        out[a:b] = _softmax_rows_times_v(s, vh)
+    return out
+
+
+def attention(q, k, v, causal: bool, scale: float, chunk: int = 256) -> np.ndarray:
+    """Full output [B, N, H_q, d] from float64 q [B,N,H_q,d], k/v [B,N,H_kv,d]."""
+    q, k, v = (np.asarray(t, dtype=np.float64) for t in (q, k, v))
+    B, N, H_q, d = q.shape
+    H_kv = k.shape[2]
+    if H_kv > H_q or k.shape != (B, N, H_kv, d) or v.shape != k.shape:
+        raise ValueError("shape mismatch")
+    out = np.empty_like(q)
+    t_all = np.arange(N)
+    for b in range(B):
+        for i in range(H_q):
+            g = group_of_head(i, H_q, H_kv)
+            kh = np.array(k[b, :, g, :])      # explicit repetition: head i's own copy
+            vh = np.array(v[b, :, g, :])
+            out[b, :, i, :] = _head_rows(q[b, :, i, :], kh, vh, t_all, causal, scale, chunk)
+    return out
+
+
+def attention_rows(q_rows, k, v, rows, N: int, causal: bool, scale: float, chunk: int = 32) -> np.ndarray:
+    """Output for selected token positions only.
+
+    ``rows`` are flat positions b*N + t; ``q_rows`` is [len(rows), H_q, d] holding
+    the query vectors of exactly those positions; k/v are the full [B,N,H_kv,d].
+    Returns [len(rows), H_q, d]. Same arithmetic as :func:`attention`.
+    """
+    q_rows = np.asarray(q_rows, dtype=np.float64)
+    rows = np.asarray(rows, dtype=np.int64)
+    B, Nk, H_kv, d = k.shape
+    assert Nk == N
+    H_q = q_rows.shape[1]
+    out = np.empty((len(rows), H_q, d), dtype=np.float64)
+    bs, ts = rows // N, rows % N
+    for b in np.unique(bs):
+        sel = np.nonzero(bs == b)[0]
+        for i in range(H_q):
+            g = group_of_head(i, H_q, H_kv)
+            kh = np.asarray(k[b, :, g, :], dtype=np.float64).copy()
+            vh = np.asarray(v[b, :, g, :], dtype=np.float64).copy()
+            out[sel, i, :] = _head_rows(q_rows[sel, i, :], kh, vh, ts[sel], causal, scale, chunk)
+    return out
+
+
+def linear(x: np.ndarray, w: np.ndarray) -> np.ndarray:
+    """y = x W^T in float64 (``nn.Linear(..., bias=False)`` with weight [out, in])."""
+    return np.asarray(x, dtype=np.float64) @ np.asarray(w, dtype=np.float64).T
+
+
+def layer(x, wq, wk, wv, wo, H_q: int, H_kv: int, d: int, causal: bool, scale: float,
+          storage_rounding: bool = True) -> np.ndarray:
+    """Full layer forward, x [B, N, d_model] -> out [B, N, d_model] (float64).
+
+    With ``storage_rounding`` the projected q, k, v and the merged attention
+    output are rounded to bf16 where a bf16 pipeline stores them; otherwise the
+    whole chain stays in float64.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    B, N, dm = x.shape
+    rnd = bf16_round if storage_rounding else (lambda a: a)
+    xf = x.reshape(B * N, dm)
+    q = rnd(linear(xf, wq)).reshape(B, N, H_q, d)
+    k = rnd(linear(xf, wk)).reshape(B, N, H_kv, d)
+    v = rnd(linear(xf, wv)).reshape(B, N, H_kv, d)
+    a = rnd(attention(q, k, v, causal, scale)).reshape(B * N, H_q * d)
+    return linear(a, wo).reshape(B, N, dm)
+
+
+def layer_rows(x, wq, wk, wv, wo, rows, H_q: int, H_kv: int, d: int, causal: bool, scale: float,
+               storage_rounding: bool = True) -> np.ndarray:
+    """Layer output at selected flat positions ``rows`` only: [len(rows), d_model].
+
+    K and V are projected for every position (attention needs all keys); Q,
+    attention and the output projection only for the selected rows.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    B, N, dm = x.shape
+    rnd = bf16_round if storage_rounding else (lambda a: a)
+    xf = x.reshape(B * N, dm)
+    rows = np.asarray(rows, dtype=np.int64)
+    k = rnd(linear(xf, wk)).reshape(B, N, H_kv, d)
+    v = rnd(linear(xf, wv)).reshape(B, N, H_kv, d)
+    q_rows = rnd(linear(xf[rows], wq)).reshape(len(rows), H_q, d)
+    a = rnd(attention_rows(q_rows, k, v, rows, N, causal, scale)).reshape(len(rows), H_q * d)
+    return linear(a, wo)
