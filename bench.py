@@ -1,0 +1,473 @@
+"""Benchmark for libsqa (decoupled-head attention on B200).
+
+Default workload (one line of JSON from rank 0): the head-configuration
+comparison at B=1, N=32768, d_head=64, non-causal, bf16 N(0,1) Q/K/V --
+MHA (16,16), GQA (16,4), MQA (16,1), SQA (8,4), sSQA (8,8), xSQA (4,4),
+xSMQA (4,1). One step runs sqa_attn_fwd once per head configuration; the
+metric is useful attention TFLOP/s = sum 4*B*N^2*H_q*d / device time.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl sqa|reference]
+                    [--workload headcfg32k|long|layer|sweep]
+
+`--impl reference` times the float64 CPU oracle on a bounded sample of the
+same workload (rank 0 only). Other workloads print extra measurement lines
+(not the headline): `long` = config N in {65536,131072,200000}, `layer` = the
+causal layer x[4,16384,2048], `sweep` = the d=128 cost grid.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+HEAD_CONFIGS_32K = [("MHA", 16, 16), ("GQA", 16, 4), ("MQA", 16, 1), ("SQA", 8, 4), ("sSQA", 8, 8),
+                    ("xSQA", 4, 4), ("xSMQA", 4, 1)]
+METRIC = "attention TFLOP/s (4*B*N^2*H_q*d, halved if causal)"
+L2_FLUSH_BYTES = 256 << 20     # > 126 MB L2
+
+
+def attn_flops(B, N, H_q, d, causal):
+    f = 4.0 * B * N * N * H_q * d
+    return f / 2 if causal else f
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            j = json.load(f)
+        return {"bf16_tflops": j["bf16_tflops"], "bf16_tflops_sustained": j.get("bf16_tflops_sustained"),
+                "hbm_gbs": j["hbm_gbs"], "source": "measured"}
+    return {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6650.0, "source": "fallback"}
+
+
+# ---------------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.dev = device_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            import torch
+            uuid = str(torch.cuda.get_device_properties(self.dev).uuid)
+            sel = ["-i", uuid if uuid.startswith("GPU-") else "GPU-" + uuid]
+        except Exception:
+            sel = ["-i", str(self.dev)]
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", *sel, "--query-gpu=" + self.FIELDS,
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.15)
+        self.proc.terminate()
+        try:
+            self.proc.wait(5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) >= 7:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+        sm = [num(r[0]) for r in rows if num(r[0]) is not None]
+        mx = [num(r[1]) for r in rows if num(r[1]) is not None]
+        pw = [num(r[2]) for r in rows if num(r[2]) is not None]
+        load = [s for s, p in zip(sm, pw) if p is not None and p > 300] or sm
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[3 + i].lower().startswith("active")})
+        return {"sm_mhz": statistics.median(load) if load else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows), "power_w_max": max(pw) if pw else None}
+
+
+# ---------------------------------------------------------------------- inputs
+def make_attn_inputs(B, N, H_q, H_kv, d, seed, factor, device, pinned_host=False):
+    import numpy as np
+    import torch
+    import synth
+    shapes = {"q": (B, N, H_q, d), "k": (B, N, H_kv, d), "v": (B, N, H_kv, d)}
+    host, dev = {}, {}
+    for name, shp in shapes.items():
+        h = torch.empty(shp, dtype=torch.bfloat16, pin_memory=pinned_host)
+        synth.fill_bf16_into(h.data_ptr(), h.numel(), seed, name, factor)
+        host[name] = h
+        dev[name] = h.to(device)
+    return host, dev
+
+
+# ---------------------------------------------------------------------- sqa arm
+def bench_sqa(args):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+    import reduced_query_head_b200 as sqa
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.gpus != world and world > 1:
+        print("warning: --gpus %d but WORLD_SIZE=%d" % (args.gpus, world), file=sys.stderr)
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=device)
+
+    peaks = load_peaks()
+    stream = torch.cuda.current_stream()
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+
+    # Each rank runs its own independent copy of the workload (weak scaling; the
+    # seed differs per rank so ranks do not compute identical problems).
+    cfgs = []
+    for name, H_q, H_kv in HEAD_CONFIGS_32K:
+        B, N, d = 1, 32768, 64
+        host, dev = make_attn_inputs(B, N, H_q, H_kv, d, rank, 1.0, device, pinned_host=True)
+        out = torch.empty((B, N, H_q, d), dtype=torch.bfloat16, device=device)
+        out_host = torch.empty((B, N, H_q, d), dtype=torch.bfloat16, pin_memory=True)
+        cfgs.append(dict(name=name, B=B, N=N, H_q=H_q, H_kv=H_kv, d=d, host=host, dev=dev, out=out,
+                         out_host=out_host, flops=attn_flops(B, N, H_q, d, False)))
+    scale = 1.0 / math.sqrt(64)
+
+    def launch(c):
+        sqa.sqa_attn_fwd(c["dev"]["q"], c["dev"]["k"], c["dev"]["v"], c["out"], c["B"], c["N"], c["H_q"],
+                         c["H_kv"], c["d"], 0, scale, stream)
+
+    # warm-up
+    for _ in range(args.warmup):
+        for c in cfgs:
+            launch(c)
+    torch.cuda.synchronize()
+    st = sqa.sqa_device_status(stream)
+    if st != sqa.SQA_OK:
+        raise RuntimeError("device status after warm-up: " + sqa.sqa_status_string(st))
+
+    # timed region: per-launch events, L2 flushed before every launch
+    ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in cfgs]
+          for _ in range(args.steps)]
+    clocks = ClockSampler(local)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    for s in range(args.steps):
+        for i, c in enumerate(cfgs):
+            flush.fill_(s & 0xFF)
+            ev[s][i][0].record(stream)
+            launch(c)
+            ev[s][i][1].record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop()
+    st = sqa.sqa_device_status(stream)
+    if st != sqa.SQA_OK:
+        raise RuntimeError("device status after timing: " + sqa.sqa_status_string(st))
+    per_cfg_ms = [[ev[s][i][0].elapsed_time(ev[s][i][1]) for s in range(args.steps)] for i in range(len(cfgs))]
+    step_ms = sum(sum(x) for x in per_cfg_ms) / args.steps
+    flops_step = sum(c["flops"] for c in cfgs)
+
+    # end to end through the same entry point, host buffers in and out
+    e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    h2d = sum(sum(t.numel() * 2 for t in c["host"].values()) for c in cfgs)
+    d2h = sum(c["out"].numel() * 2 for c in cfgs)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    for s in range(args.steps):
+        flush.fill_((s + 1) & 0xFF)
+        e2e_ev[s][0].record(stream)
+        for c in cfgs:
+            for name in ("q", "k", "v"):
+                c["dev"][name].copy_(c["host"][name], non_blocking=True)
+            launch(c)
+            c["out_host"].copy_(c["out"], non_blocking=True)
+        e2e_ev[s][1].record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = sum(a.elapsed_time(b) for a, b in e2e_ev) / args.steps
+
+    t_local = torch.tensor([step_ms, e2e_ms], dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(t_local, op=dist.ReduceOp.MAX)
+    step_ms_max, e2e_ms_max = float(t_local[0]), float(t_local[1])
+
+    value = flops_step * world / (step_ms_max * 1e-3) / 1e12
+    e2e_value = flops_step * world / (e2e_ms_max * 1e-3) / 1e12
+    launch_ms = step_ms / len(cfgs)
+    achieved = (flops_step / len(cfgs)) / (launch_ms * 1e-3) / 1e12
+    peak = peaks["bf16_tflops"]
+
+    result = None
+    if rank == 0:
+        cpu = cpu_baseline(seconds=args.cpu_seconds) if (world == 1 and not args.no_cpu_baseline) else None
+        per = {}
+        for i, c in enumerate(cfgs):
+            ms = statistics.median(per_cfg_ms[i])
+            per[c["name"]] = {"H_q": c["H_q"], "H_kv": c["H_kv"], "ms_median": round(ms, 4),
+                              "ms_min": round(min(per_cfg_ms[i]), 4),
+                              "tflops": round(c["flops"] / (ms * 1e-3) / 1e12, 1)}
+        t16 = statistics.mean([per[n]["ms_median"] for n in ("MHA", "GQA", "MQA")])
+        t8 = statistics.mean([per[n]["ms_median"] for n in ("SQA", "sSQA")])
+        t4 = statistics.mean([per[n]["ms_median"] for n in ("xSQA", "xSMQA")])
+        result = {
+            "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(step_ms_max, 4),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded N(0,1) bf16 Q/K/V; per-rank seed)",
+            "config": {"workload": "head-config comparison, B=1 N=32768 d_head=64 non-causal "
+                                   "(MHA 16/16, GQA 16/4, MQA 16/1, SQA 8/4, sSQA 8/8, xSQA 4/4, xSMQA 4/1)",
+                       "global_batch": world, "seq_len": 32768, "parallelism": "dp%d" % world,
+                       "l2": "flushed (256 MiB write) before every timed launch"},
+            "pct_of_peak": round(100.0 * value / world / peak, 1),
+            "roofline": {"bound": "tensor", "kernel": "sqa::attn_fwd_kernel<64>", "achieved": round(achieved, 1),
+                         "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 3),
+                         "peak_source": peaks["source"] + " bf16 dense (burst; each launch timed alone)",
+                         "traffic": args.traffic},
+            "e2e": {"value": round(e2e_value, 2), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms_max, 4)},
+            "gpu_launches": args.steps * len(cfgs),
+            "clocks": clk,
+            "per_config": per,
+            "speedup_vs_flop_ratio": {"t16/t8": round(t16 / t8, 3), "flop_ratio_16/8": 2.0,
+                                      "t16/t4": round(t16 / t4, 3), "flop_ratio_16/4": 4.0},
+            "cpu_baseline": cpu,
+        }
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return result
+
+
+# ---------------------------------------------------------------------- oracle timing
+def _blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        info = threadpool_info()
+        return max([i.get("num_threads", 1) for i in info] or [os.cpu_count() or 1])
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def oracle_sample(rows_per_cfg, seed=0):
+    """Oracle on `rows_per_cfg` query positions (all heads) of every head config.
+    Returns (useful flops, seconds)."""
+    import numpy as np
+    import oracle
+    import synth
+    N, d = 32768, 64
+    flops, secs = 0.0, 0.0
+    for name, H_q, H_kv in HEAD_CONFIGS_32K:
+        kb = synth.bf16_bits((1, N, H_kv, d), seed, "k")
+        vb = synth.bf16_bits((1, N, H_kv, d), seed, "v")
+        rows = synth.sample_rows(rows_per_cfg, N, seed ^ 0x5A17)
+        q = np.empty((len(rows), H_q, d), dtype=np.uint16)
+        full_q = synth.bf16_bits((1, N, H_q, d), seed, "q").reshape(N, H_q, d)
+        q[:] = full_q[rows]
+        t0 = time.perf_counter()
+        oracle.attention_rows(oracle.widen_bf16(q), oracle.widen_bf16(kb), oracle.widen_bf16(vb), rows, N,
+                              False, 1.0 / math.sqrt(d))
+        secs += time.perf_counter() - t0
+        flops += 4.0 * len(rows) * N * H_q * d
+    return flops, secs
+
+
+def cpu_baseline(seconds=15.0):
+    # size the sample from a short probe so the whole leg takes ~`seconds`
+    f0, s0 = oracle_sample(8)
+    rows = int(max(8, min(4096, 8 * seconds / max(s0, 1e-3))))
+    f, s = oracle_sample(rows)
+    return {"value": round(f / s / 1e12, 6), "unit": "TFLOP/s", "cores": _blas_threads(), "kind": "oracle",
+            "sample": "%d query positions (all heads) of each of the 7 head configs at N=32768, d=64, "
+                      "float64 numpy/BLAS; %.1f s" % (rows, s)}
+
+
+def bench_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return None
+    rows = 16
+    for _ in range(args.warmup):
+        oracle_sample(rows)
+    f_tot, s_tot = 0.0, 0.0
+    for s in range(args.steps):
+        f, t = oracle_sample(rows, seed=s)
+        f_tot += f
+        s_tot += t
+    value = f_tot / s_tot / 1e12
+    cores = _blas_threads()
+    sample = "%d query positions (all heads) of each of the 7 head configs per step, float64 oracle" % rows
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s",
+        "n_gpus": int(os.environ.get("WORLD_SIZE", "1")), "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(1e3 * s_tot / args.steps, 3), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded N(0,1) bf16 Q/K/V)",
+        "config": {"workload": "head-config comparison, B=1 N=32768 d_head=64 non-causal (sampled rows)",
+                   "global_batch": 1, "seq_len": 32768, "parallelism": "none (host cores)"},
+        "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+# ---------------------------------------------------------------------- extra workloads
+def _time_launches(fn, reps, flush, stream):
+    import torch
+    evs = []
+    for r in range(reps):
+        flush.fill_(r & 0xFF)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        fn()
+        b.record(stream)
+        evs.append((a, b))
+    torch.cuda.synchronize()
+    return [a.elapsed_time(b) for a, b in evs]
+
+
+def bench_extra(args):
+    import torch
+    import reduced_query_head_b200 as sqa
+    device = torch.device("cuda", 0)
+    stream = torch.cuda.current_stream()
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+    peaks = load_peaks()
+    lines = []
+    if args.workload in ("long", "sweep"):
+        if args.workload == "long":
+            grid = [(N, H_q, H_kv, 64, c, 1.0, 0) for N in (65536, 131072, 200000)
+                    for (_, H_q, H_kv) in (("MHA", 16, 16), ("SQA", 8, 4), ("xSQA", 4, 4)) for c in (0,)]
+        else:
+            grid = []
+            idx = 0
+            for N in (32768, 65536, 131072, 200000):
+                for H_q in (32, 16, 8, 4):
+                    for H_kv in (8, 4, 1):
+                        if H_kv <= H_q:
+                            for c in (0, 1):
+                                grid.append((N, H_q, H_kv, 128, c, 0.5, idx))
+                            idx += 1
+        for N, H_q, H_kv, d, causal, factor, seed in grid:
+            _, dev = make_attn_inputs(1, N, H_q, H_kv, d, seed, factor, device)
+            out = torch.empty((1, N, H_q, d), dtype=torch.bfloat16, device=device)
+
+            def fn():
+                sqa.sqa_attn_fwd(dev["q"], dev["k"], dev["v"], out, 1, N, H_q, H_kv, d, causal, d ** -0.5, stream)
+            for _ in range(args.warmup):
+                fn()
+            ms = _time_launches(fn, args.steps, flush, stream)
+            assert sqa.sqa_device_status(stream) == 0
+            fl = attn_flops(1, N, H_q, d, causal)
+            med = statistics.median(ms)
+            lines.append({"workload": args.workload, "N": N, "H_q": H_q, "H_kv": H_kv, "d": d, "causal": causal,
+                          "ms_median": round(med, 3), "ms_min": round(min(ms), 3),
+                          "tflops": round(fl / (med * 1e-3) / 1e12, 1),
+                          "pct_of_peak": round(100 * fl / (med * 1e-3) / 1e12 / peaks["bf16_tflops"], 1)})
+            print(json.dumps(lines[-1]), flush=True)
+            del dev, out
+    elif args.workload == "layer":
+        import synth
+        B, N, dm, H_q, H_kv, d = 4, 16384, 2048, 16, 8, 64
+        M = B * N
+
+        def mk(shape, name, factor):
+            h = torch.empty(shape, dtype=torch.bfloat16)
+            synth.fill_bf16_into(h.data_ptr(), h.numel(), 0, name, factor)
+            return h.to(device)
+        x = mk((B, N, dm), "x", 1.0)
+        wq, wk, wv = mk((H_q * d, dm), "wq", 0.02), mk((H_kv * d, dm), "wk", 0.02), mk((H_kv * d, dm), "wv", 0.02)
+        wo = mk((dm, H_q * d), "wo", 0.02)
+        out = torch.empty((B, N, dm), dtype=torch.bfloat16, device=device)
+        ws_bytes = sqa.sqa_layer_workspace_bytes(B, N, dm, H_q, H_kv, d)
+        ws = torch.empty(ws_bytes, dtype=torch.uint8, device=device)
+
+        def fn():
+            sqa.sqa_layer_fwd(x, wq, wk, wv, wo, out, ws, ws_bytes, B, N, dm, H_q, H_kv, d, 1, 0.125, stream)
+        for _ in range(args.warmup):
+            fn()
+        ms = _time_launches(fn, args.steps, flush, stream)
+        assert sqa.sqa_device_status(stream) == 0
+        fl_attn = attn_flops(B, N, H_q, d, True)
+        fl_gemm = 2.0 * M * dm * (H_q + 2 * H_kv) * d + 2.0 * M * (H_q * d) * dm
+        med = statistics.median(ms)
+        # per-kernel split
+        Q = ws[:0]
+        qkv = torch.empty((M, (H_q + 2 * H_kv) * d), dtype=torch.bfloat16, device=device)
+        wqkv = torch.cat([wq, wk, wv], 0).contiguous()
+        ms_qkv = statistics.median(_time_launches(
+            lambda: sqa.sqa_linear_fwd(x, wqkv, qkv, M, dm, (H_q + 2 * H_kv) * d, stream), args.steps, flush, stream))
+        a = torch.empty((M, H_q * d), dtype=torch.bfloat16, device=device)
+        ms_o = statistics.median(_time_launches(
+            lambda: sqa.sqa_linear_fwd(a, wo, out, M, H_q * d, dm, stream), args.steps, flush, stream))
+        lines.append({"workload": "layer", "ms_per_layer": round(med, 3), "tflops_total":
+                      round((fl_attn + fl_gemm) / (med * 1e-3) / 1e12, 1), "ms_qkv_gemm": round(ms_qkv, 3),
+                      "qkv_gemm_tflops": round(2.0 * M * dm * (H_q + 2 * H_kv) * d / (ms_qkv * 1e-3) / 1e12, 1),
+                      "ms_o_gemm": round(ms_o, 3),
+                      "o_gemm_tflops": round(2.0 * M * (H_q * d) * dm / (ms_o * 1e-3) / 1e12, 1),
+                      "ms_attention_est": round(med - ms_qkv - ms_o, 3)})
+        print(json.dumps(lines[-1]), flush=True)
+    return lines
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["sqa", "reference"], default="sqa")
+    ap.add_argument("--workload", choices=["headcfg32k", "long", "layer", "sweep"], default="headcfg32k")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--traffic", type=float, default=None,
+                    help="ncu dram bytes per attention launch, if captured for this kernel build")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "sqa":
+        print("note: raising --warmup to 3", file=sys.stderr)
+        args.warmup = 3
+    if args.impl == "reference":
+        r = bench_reference(args)
+        if r is not None:
+            print(json.dumps(r), flush=True)
+        return
+    if args.workload != "headcfg32k":
+        bench_extra(args)
+        return
+    r = bench_sqa(args)
+    if r is not None:
+        print(json.dumps(r), flush=True)
+
+
+if __name__ == "__main__":
+    main()

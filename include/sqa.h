@@ -1,0 +1,131 @@
+/*
+ * libsqa -- full-sequence attention with decoupled query / key-value head
+ * counts on NVIDIA B200 (sm_100a).
+ *
+ * The operation (definitions restated from the pages this library follows):
+ *
+ *   Query head i in [0, H_q) reads key/value group g(i) = floor(i * H_kv / H_q),
+ *   so contiguous blocks of query heads share one group. G = H is multi-head
+ *   attention, G = 1 multi-query attention, 1 < G < H grouped-query attention
+ *   (GQA explainer, "MHA・MQA・GQAの関係" equations and head-to-group diagram).
+ *   Sparse Query Attention uses fewer query heads than the base head count,
+ *   which cuts the score and value FLOPs in proportion ("Sparse Query Attention
+ *   (SQA)", abstract). The attention of one head is
+ *     out[t] = sum_u softmax_u(scale * q[t] . k[u]) v[u]
+ *   over all keys u, or over u <= t when causal (the GQA module's
+ *   scaled_dot_product_attention(..., is_causal=True)).
+ *
+ * Conventions for every entry point:
+ *   - Tensor pointers are caller-owned DEVICE pointers to contiguous bf16 data,
+ *     16-byte aligned. The library never frees or keeps them.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t, NULL = legacy default
+ *     stream) and return after the work is enqueued.
+ *   - Argument errors are detected on the host before anything is launched
+ *     and returned as an sqa_status; nothing is written in that case.
+ *   - Device-side failures (a bounded wait inside a kernel that ran out) are
+ *     recorded in a per-device status word and reported by sqa_device_status().
+ *   - The library allocates no device memory per call; the layer takes a
+ *     caller-provided workspace.
+ *   - Thread-safe; each call may target any device (the current one is used).
+ */
+#ifndef SQA_H
+#define SQA_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  SQA_OK = 0,
+  SQA_ERR_INVALID_ARG = 1,  /* null/misaligned pointer, bad size, bad scale */
+  SQA_ERR_UNSUPPORTED = 2,  /* valid request this build does not implement (e.g. d_head) */
+  SQA_ERR_CUDA = 3,         /* a CUDA runtime/driver call failed */
+  SQA_ERR_TIMEOUT = 4,      /* a kernel wait exceeded its limit (device status) */
+  SQA_ERR_WORKSPACE = 5     /* workspace too small or misaligned */
+} sqa_status;
+
+/*
+ * Attention core.
+ *   q   [B, N, H_q,  d_head]   (the [B, T, H, d] view of the GQA module)
+ *   k   [B, N, H_kv, d_head]
+ *   v   [B, N, H_kv, d_head]
+ *   out [B, N, H_q,  d_head]   written in full
+ * Requirements: B, N >= 1; 1 <= H_kv <= H_q; d_head in {64, 128};
+ * scale finite and > 0 (1/sqrt(d_head) gives the SDPA default); causal in {0,1}.
+ * Arithmetic: bf16 inputs, fp32 accumulation and softmax, bf16 output.
+ * Returns SQA_OK once the kernel is enqueued.
+ */
+int sqa_attn_fwd(const void* q, const void* k, const void* v, void* out,
+                 int B, int N, int H_q, int H_kv, int d_head,
+                 int causal, float scale, void* stream);
+
+/*
+ * Bytes of device workspace sqa_layer_fwd needs (Q, K, V and the merged
+ * attention output, each 256-byte aligned). Returns 0 for invalid sizes.
+ */
+size_t sqa_layer_workspace_bytes(int B, int N, int d_model, int H_q, int H_kv, int d_head);
+
+/*
+ * Attention layer forward (the GQA explainer's module, "PyTorchでのGQA実装",
+ * with H_q query heads and H_kv key/value groups, no biases):
+ *   Q = x Wq^T, K = x Wk^T, V = x Wv^T   viewed [B, N, H, d_head]
+ *   A = attention(Q, K, V)               merged back to [B, N, H_q * d_head]
+ *   out = A Wo^T
+ *   x   [B, N, d_model]
+ *   Wq  [H_q * d_head,  d_model]   (nn.Linear weight layout [out, in])
+ *   Wk  [H_kv * d_head, d_model]
+ *   Wv  [H_kv * d_head, d_model]
+ *   Wo  [d_model, H_q * d_head]
+ *   out [B, N, d_model]
+ *   workspace: device memory of at least sqa_layer_workspace_bytes(...),
+ *   256-byte aligned; its contents are scratch and are overwritten.
+ * Requirements: as sqa_attn_fwd, plus d_model >= 8 and d_model % 8 == 0.
+ * Q, K and V are stored in bf16 between the kernels, as is A.
+ */
+int sqa_layer_fwd(const void* x, const void* Wq, const void* Wk, const void* Wv, const void* Wo,
+                  void* out, void* workspace, size_t workspace_bytes,
+                  int B, int N, int d_model, int H_q, int H_kv, int d_head,
+                  int causal, float scale, void* stream);
+
+/*
+ * Plain projection y[M, N_out] = x[M, K] W[N_out, K]^T (bf16 in, fp32
+ * accumulate, bf16 out): the layer's linear step exposed on its own.
+ * Requirements: M >= 1, K >= 8, K % 8 == 0, N_out >= 8, N_out % 8 == 0.
+ */
+int sqa_linear_fwd(const void* x, const void* W, void* y, long long M, int K, int N_out, void* stream);
+
+/*
+ * Synchronises `stream`, then returns and clears the current device's status
+ * word: SQA_OK, or SQA_ERR_TIMEOUT if any kernel gave up on a wait since the
+ * last call. SQA_ERR_CUDA if the synchronisation itself failed.
+ */
+int sqa_device_status(void* stream);
+
+/*
+ * Upper limit (nanoseconds) on each wait inside the kernels of later calls on
+ * this device; 0 restores the default (2 s). Returns the previous value.
+ */
+unsigned long long sqa_set_wait_limit_ns(unsigned long long ns);
+
+/*
+ * Diagnostic: launches one warp that waits on a shared-memory barrier nothing
+ * ever completes, through the same bounded wait the kernels use, with the
+ * given limit (nanoseconds, 1e3..1e10). Synchronises `stream` and returns the
+ * status the device recorded -- SQA_ERR_TIMEOUT when the bound works -- and
+ * clears it. Shows that a stuck wait ends with a status instead of a hang.
+ */
+int sqa_check_wait_timeout(unsigned long long limit_ns, void* stream);
+
+/* Human-readable name of a status code (static string). */
+const char* sqa_status_string(int status);
+
+/* Library version, major*10000 + minor*100 + patch. */
+int sqa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SQA_H */

@@ -96,10 +96,13 @@ def _head_rows(qh, kh, vh, t_idx, causal, scale, chunk):
     keys = np.arange(N)
     for a in range(0, qh.shape[0], chunk):
         b = min(a + chunk, qh.shape[0])
-        s = scale * (qh[a:b] @ kh.T)              # explicit score rows
+        # keys past the chunk's last causal position are masked for every row
+        # of the chunk, so they are left out of the row instead of set to -inf
+        n = min(N, int(t_idx[a:b].max()) + 1) if causal else N
+        s = scale * (qh[a:b] @ kh[:n].T)          # explicit score rows
         if causal:
-            s[keys[None, :] > t_idx[a:b, None]] = -np.inf
-        out[a:b] = _softmax_rows_times_v(s, vh)
+            s[keys[None, :n] > t_idx[a:b, None]] = -np.inf
+        out[a:b] = _softmax_rows_times_v(s, vh[:n])
     return out
 
 

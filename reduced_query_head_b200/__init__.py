@@ -1,0 +1,130 @@
+"""Python binding for libsqa (decoupled-head attention on B200 / sm_100a).
+
+Argument marshalling only: every step runs in the CUDA kernels of
+``libsqa.so``. The functions take torch CUDA tensors (bf16, contiguous) or raw
+device pointers, and the current torch CUDA stream unless one is given. There
+is no fallback: if the library is missing, importing this package raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+from .build import LIB as _LIB_PATH
+
+__all__ = [
+    "SQA_OK", "SQA_ERR_INVALID_ARG", "SQA_ERR_UNSUPPORTED", "SQA_ERR_CUDA", "SQA_ERR_TIMEOUT",
+    "SQA_ERR_WORKSPACE", "SqaError", "lib", "EXPORTED_SYMBOLS", "sqa_attn_fwd", "sqa_layer_fwd",
+    "sqa_layer_workspace_bytes", "sqa_linear_fwd", "sqa_device_status", "sqa_set_wait_limit_ns",
+    "sqa_check_wait_timeout", "sqa_status_string", "sqa_version",
+]
+
+SQA_OK, SQA_ERR_INVALID_ARG, SQA_ERR_UNSUPPORTED, SQA_ERR_CUDA, SQA_ERR_TIMEOUT, SQA_ERR_WORKSPACE = range(6)
+
+EXPORTED_SYMBOLS = (
+    "sqa_attn_fwd", "sqa_layer_workspace_bytes", "sqa_layer_fwd", "sqa_linear_fwd", "sqa_device_status",
+    "sqa_set_wait_limit_ns", "sqa_check_wait_timeout", "sqa_status_string", "sqa_version",
+)
+
+if not os.path.exists(_LIB_PATH):
+    raise ImportError(
+        "libsqa.so is not built (expected at %s); run `python -m reduced_query_head_b200.build`" % _LIB_PATH)
+
+lib = ctypes.CDLL(_LIB_PATH)
+
+_vp, _i, _f, _sz, _ll, _ull = (ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t,
+                               ctypes.c_longlong, ctypes.c_ulonglong)
+lib.sqa_attn_fwd.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _vp]
+lib.sqa_attn_fwd.restype = _i
+lib.sqa_layer_workspace_bytes.argtypes = [_i, _i, _i, _i, _i, _i]
+lib.sqa_layer_workspace_bytes.restype = _sz
+lib.sqa_layer_fwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _i, _i, _i, _i, _i, _i, _i, _f, _vp]
+lib.sqa_layer_fwd.restype = _i
+lib.sqa_linear_fwd.argtypes = [_vp, _vp, _vp, _ll, _i, _i, _vp]
+lib.sqa_linear_fwd.restype = _i
+lib.sqa_device_status.argtypes = [_vp]
+lib.sqa_device_status.restype = _i
+lib.sqa_set_wait_limit_ns.argtypes = [_ull]
+lib.sqa_set_wait_limit_ns.restype = _ull
+lib.sqa_check_wait_timeout.argtypes = [_ull, _vp]
+lib.sqa_check_wait_timeout.restype = _i
+lib.sqa_status_string.argtypes = [_i]
+lib.sqa_status_string.restype = ctypes.c_char_p
+lib.sqa_version.argtypes = []
+lib.sqa_version.restype = _i
+
+
+class SqaError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        super().__init__("%s failed: %s" % (what, sqa_status_string(status)))
+        self.status = status
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    if not t.is_cuda:
+        raise ValueError("expected a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError("expected a contiguous tensor")
+    return t.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _check(status: int, what: str, raise_on_error: bool):
+    if raise_on_error and status != SQA_OK:
+        raise SqaError(status, what)
+    return status
+
+
+def sqa_attn_fwd(q, k, v, out, B, N, H_q, H_kv, d_head, causal, scale, stream=None, raise_on_error=True):
+    st = lib.sqa_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), B, N, H_q, H_kv, d_head, int(causal),
+                          float(scale), _stream(stream))
+    return _check(st, "sqa_attn_fwd", raise_on_error)
+
+
+def sqa_layer_workspace_bytes(B, N, d_model, H_q, H_kv, d_head):
+    return int(lib.sqa_layer_workspace_bytes(B, N, d_model, H_q, H_kv, d_head))
+
+
+def sqa_layer_fwd(x, Wq, Wk, Wv, Wo, out, workspace, workspace_bytes, B, N, d_model, H_q, H_kv, d_head, causal,
+                  scale, stream=None, raise_on_error=True):
+    st = lib.sqa_layer_fwd(_ptr(x), _ptr(Wq), _ptr(Wk), _ptr(Wv), _ptr(Wo), _ptr(out), _ptr(workspace),
+                           int(workspace_bytes), B, N, d_model, H_q, H_kv, d_head, int(causal), float(scale),
+                           _stream(stream))
+    return _check(st, "sqa_layer_fwd", raise_on_error)
+
+
+def sqa_linear_fwd(x, W, y, M, K, N_out, stream=None, raise_on_error=True):
+    st = lib.sqa_linear_fwd(_ptr(x), _ptr(W), _ptr(y), M, K, N_out, _stream(stream))
+    return _check(st, "sqa_linear_fwd", raise_on_error)
+
+
+def sqa_device_status(stream=None):
+    return int(lib.sqa_device_status(_stream(stream)))
+
+
+def sqa_set_wait_limit_ns(ns: int) -> int:
+    return int(lib.sqa_set_wait_limit_ns(int(ns)))
+
+
+def sqa_check_wait_timeout(limit_ns: int, stream=None) -> int:
+    return int(lib.sqa_check_wait_timeout(int(limit_ns), _stream(stream)))
+
+
+def sqa_status_string(status: int) -> str:
+    return lib.sqa_status_string(int(status)).decode()
+
+
+def sqa_version() -> int:
+    return int(lib.sqa_version())

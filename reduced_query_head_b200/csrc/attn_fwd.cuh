@@ -1,0 +1,354 @@
+// Forward attention with decoupled head counts on sm_100a.
+//
+// out[b,t,i,:] = softmax_u(scale * q[b,t,i,:] . k[b,u,g(i),:]) v[b,u,g(i),:],
+// g(i) = floor(i * H_kv / H_q), keys u in [0, N) or u <= t when causal.
+// This is scaled-dot-product attention with per-group key/value sharing as in
+// the GQA explainer ("MHA・MQA・GQAの関係" equations and the head-to-group
+// diagram); Sparse Query Attention is the same computation with fewer query
+// heads ("Sparse Query Attention (SQA)", abstract).
+//
+// One CTA owns two 128-row query tiles of one (batch, head block). A head
+// block is P consecutive query heads of one KV group (P a power of two
+// dividing H_q/H_kv), stacked so that tile row r = token_local * P + head
+// offset: every key/value tile brought into shared memory serves all P heads.
+//
+// Warp roles (12 warps):
+//   warp 0   TMA producer: Q0/Q1 once, then K_j and V_j into a ring of stages
+//   warp 1   MMA issuer: S_k = Q_k K_j^T into TMEM, O_k += P_k V_j from TMEM
+//   warp 2   owns the TMEM allocation
+//   warps 4-7 / 8-11  softmax for tile 0 / tile 1 (thread = row = TMEM lane):
+//            online softmax with a lazily rescaled running max, P written
+//            back to TMEM as bf16 over S, epilogue O / l -> bf16 -> global.
+//
+// TMEM columns: S0 [0,128), S1 [128,256), O0 [256,256+D), O1 [256+D,256+2D).
+// Every wait is bounded; on time-out the kernel records the status, drains
+// its own copies and MMAs, frees TMEM and returns.
+#pragma once
+
+#include "sm100.cuh"
+
+namespace sqa {
+
+struct AttnParams {
+  __nv_bfloat16* out;   // [B, N, H_q, D]
+  int B, N, H_q, H_kv;
+  int P, log2P;         // heads stacked per tile
+  int tpt;              // tokens per 128-row tile = 128 / P
+  int n_pairs;          // tile pairs per (batch, head block)
+  int n_hb;             // head blocks = H_q / P
+  int causal;
+  float scale_log2;     // scale * log2(e)
+  int* status;
+  unsigned long long timeout_ns;
+};
+
+template <int D>
+struct AttnCfg {
+  static constexpr int BM = 128;
+  static constexpr int BN = 128;
+  static constexpr int KCH = D / 64;                    // 128-byte column chunks
+  static constexpr int STAGES = (D == 64) ? 4 : 2;
+  static constexpr int Q_BYTES = BM * D * 2;            // one Q tile
+  static constexpr int KV_BYTES = BN * D * 2;           // one K (or V) tile
+  static constexpr int CHUNK_Q = BM * 128;              // bytes per column chunk
+  static constexpr int CHUNK_KV = BN * 128;
+  // shared-memory map (offsets from a 1024-aligned base)
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_K = OFF_Q + 2 * Q_BYTES;
+  static constexpr int OFF_V = OFF_K + STAGES * KV_BYTES;
+  static constexpr int OFF_BAR = OFF_V + STAGES * KV_BYTES;
+  // barriers: q_full, k_full[S], v_full[S], kv_empty[S], s_full[2], p_full[2], o_full[2], drain
+  static constexpr int BAR_Q = 0;
+  static constexpr int BAR_KF = 1;
+  static constexpr int BAR_VF = BAR_KF + STAGES;
+  static constexpr int BAR_KVE = BAR_VF + STAGES;
+  static constexpr int BAR_S = BAR_KVE + STAGES;
+  static constexpr int BAR_P = BAR_S + 2;
+  static constexpr int BAR_O = BAR_P + 2;
+  static constexpr int BAR_DRAIN = BAR_O + 2;
+  static constexpr int N_BARS = BAR_DRAIN + 1;
+  static constexpr int OFF_MISC = OFF_BAR + N_BARS * 8;  // tmem base (u32), abort flag (u32)
+  static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;  // + alignment slack
+  static constexpr int THREADS = 384;
+  static constexpr uint32_t TMEM_COLS = 512;
+  static constexpr uint32_t COL_S0 = 0, COL_S1 = 128, COL_O0 = 256, COL_O1 = 256 + D;
+};
+
+template <int D>
+__global__ void __launch_bounds__(384, 1)
+    attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                    const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
+  using C = AttnCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+  uint32_t* misc = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
+  volatile uint32_t* tmem_slot = misc;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 1);
+  auto bar = [&](int i) { return smem_u32(&bars[i]); };
+
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5;
+  const int lane = tid & 31;
+
+  // ---- work item (longest first when causal)
+  const int per_pair = p.n_hb * p.B;
+  int qp = blockIdx.x / per_pair;
+  const int rest = blockIdx.x - qp * per_pair;
+  if (p.causal) qp = p.n_pairs - 1 - qp;
+  const int hb = rest % p.n_hb;
+  const int b = rest / p.n_hb;
+  const int head0 = hb * p.P;
+  const int g = (int)(((long long)head0 * p.H_kv) / p.H_q);
+  const int n_kv_all = (p.N + C::BN - 1) / C::BN;
+  int t0[2], n_kv[2];
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+    t0[k] = (qp * 2 + k) * p.tpt;
+    if (t0[k] >= p.N) {
+      n_kv[k] = 0;
+    } else if (p.causal) {
+      const int last = min(t0[k] + p.tpt - 1, p.N - 1);
+      n_kv[k] = last / C::BN + 1;
+    } else {
+      n_kv[k] = n_kv_all;
+    }
+  }
+  const int n_max = max(n_kv[0], n_kv[1]);
+
+  WaitCtl ctl{abort_flag, p.status, p.timeout_ns};
+
+  if (tid == 0) {
+    for (int i = 0; i < C::N_BARS; ++i) mbar_init(bar(i), (i == C::BAR_P || i == C::BAR_P + 1) ? 4 : 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 2) {
+    tmem_alloc(smem_u32((const void*)tmem_slot), C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ======================= TMA producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+      mbar_arrive_expect_tx(bar(C::BAR_Q), 2 * C::Q_BYTES);
+#pragma unroll
+      for (int k = 0; k < 2; ++k)
+#pragma unroll
+        for (int c = 0; c < C::KCH; ++c)
+          tma_load_4d(sbase + C::OFF_Q + k * C::Q_BYTES + c * C::CHUNK_Q, &tm_q, bar(C::BAR_Q), c * 64, head0,
+                      t0[k], b);
+      int filled = 0;
+      for (int j = 0; j < n_max; ++j) {
+        const int s = j % C::STAGES;
+        const int round = j / C::STAGES;
+        if (round > 0 && !mbar_wait(bar(C::BAR_KVE + s), (round - 1) & 1, ctl)) break;
+        mbar_arrive_expect_tx(bar(C::BAR_KF + s), C::KV_BYTES);
+#pragma unroll
+        for (int c = 0; c < C::KCH; ++c)
+          tma_load_4d(sbase + C::OFF_K + s * C::KV_BYTES + c * C::CHUNK_KV, &tm_k, bar(C::BAR_KF + s), c * 64, g,
+                      j * C::BN, b);
+        mbar_arrive_expect_tx(bar(C::BAR_VF + s), C::KV_BYTES);
+#pragma unroll
+        for (int c = 0; c < C::KCH; ++c)
+          tma_load_4d(sbase + C::OFF_V + s * C::KV_BYTES + c * C::CHUNK_KV, &tm_v, bar(C::BAR_VF + s), c * 64, g,
+                      j * C::BN, b);
+        filled = j + 1;
+      }
+      // Drain: wait (bounded) for the copies this thread issued, so none lands after exit.
+      WaitCtl drain{abort_flag, p.status, p.timeout_ns};
+      volatile int zero = 0;
+      drain.abort_flag = &zero;
+      mbar_wait(bar(C::BAR_Q), 0, drain);
+      for (int j = max(0, filled - C::STAGES); j < filled; ++j) {
+        const int s = j % C::STAGES;
+        mbar_wait(bar(C::BAR_KF + s), (j / C::STAGES) & 1, drain);
+        mbar_wait(bar(C::BAR_VF + s), (j / C::STAGES) & 1, drain);
+      }
+    }
+  } else if (warp == 1) {
+    // ======================= MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t IDESC_S = idesc_bf16_f32(C::BM, C::BN, 0, 0);
+      constexpr uint32_t IDESC_O = idesc_bf16_f32(C::BM, D, 0, 1);
+      const uint32_t col_s[2] = {C::COL_S0, C::COL_S1};
+      const uint32_t col_o[2] = {C::COL_O0, C::COL_O1};
+      bool ok = mbar_wait(bar(C::BAR_Q), 0, ctl);
+      auto issue_s = [&](int k, int s) {
+        const uint32_t qa = sbase + C::OFF_Q + k * C::Q_BYTES;
+        const uint32_t ka = sbase + C::OFF_K + s * C::KV_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * C::CHUNK_Q + (kk & 3) * 32;
+          const uint32_t offk = (kk >> 2) * C::CHUNK_KV + (kk & 3) * 32;
+          umma_ss(tmem + col_s[k], sdesc_sw128(qa + off, 16, 1024), sdesc_sw128(ka + offk, 16, 1024), IDESC_S,
+                  kk > 0);
+        }
+      };
+      auto issue_pv = [&](int k, int s, int j) {
+        const uint32_t va = sbase + C::OFF_V + s * C::KV_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < C::BN / 16; ++kk) {
+          umma_ts(tmem + col_o[k], tmem + col_s[k] + kk * 8, sdesc_sw128(va + kk * 16 * 128, C::CHUNK_KV, 1024),
+                  IDESC_O, (j > 0 || kk > 0) ? 1u : 0u);
+        }
+      };
+      if (ok && n_max > 0) {
+        ok = mbar_wait(bar(C::BAR_KF + 0), 0, ctl);
+        if (ok) {
+          tc_fence_after();
+          for (int k = 0; k < 2; ++k)
+            if (n_kv[k] > 0) {
+              issue_s(k, 0);
+              umma_commit(bar(C::BAR_S + k));
+            }
+        }
+      }
+      for (int j = 0; ok && j < n_max; ++j) {
+        const int s = j % C::STAGES;
+        const uint32_t ph = (j / C::STAGES) & 1;
+        const int s1 = (j + 1) % C::STAGES;
+        const uint32_t ph1 = ((j + 1) / C::STAGES) & 1;
+        if (!mbar_wait(bar(C::BAR_VF + s), ph, ctl)) { ok = false; break; }
+        for (int k = 0; k < 2 && ok; ++k) {
+          if (j >= n_kv[k]) continue;
+          if (!mbar_wait(bar(C::BAR_P + k), j & 1, ctl)) { ok = false; break; }
+          tc_fence_after();
+          issue_pv(k, s, j);
+          if (j == n_kv[k] - 1) {
+            umma_commit(bar(C::BAR_O + k));
+          } else {
+            if (!mbar_wait(bar(C::BAR_KF + s1), ph1, ctl)) { ok = false; break; }
+            tc_fence_after();
+            issue_s(k, s1);
+            umma_commit(bar(C::BAR_S + k));
+          }
+        }
+        umma_commit(bar(C::BAR_KVE + s));
+      }
+      // Drain: every MMA issued above has finished before TMEM is released.
+      umma_commit(bar(C::BAR_DRAIN));
+      WaitCtl drain{abort_flag, p.status, p.timeout_ns};
+      volatile int zero = 0;
+      drain.abort_flag = &zero;
+      mbar_wait(bar(C::BAR_DRAIN), 0, drain);
+    }
+  } else if (warp >= 4) {
+    // ======================= softmax + epilogue, one thread per tile row
+    const int k = (warp - 4) >> 2;
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;
+    const uint32_t lane_base = tmem + (uint32_t(quarter * 32) << 16);
+    const uint32_t s_addr = lane_base + (k ? C::COL_S1 : C::COL_S0);
+    const uint32_t o_addr = lane_base + (k ? C::COL_O1 : C::COL_O0);
+    const int token = t0[k] + (row >> p.log2P);
+    const int head = head0 + (row & (p.P - 1));
+    const float sl2 = p.scale_log2;
+    const int nk = n_kv[k];
+    const int t_first = t0[k];
+    float m = -INFINITY, l = 0.f;
+    bool ok = true;
+    for (int j = 0; j < nk; ++j) {
+      if (!mbar_wait_warp(bar(C::BAR_S + k), j & 1, ctl)) { ok = false; break; }
+      tc_fence_after();
+      float s[128];
+      {
+        uint32_t r[64];
+        tmem_ld64(s_addr, r);
+#pragma unroll
+        for (int u = 0; u < 64; ++u) s[u] = __uint_as_float(r[u]);
+        tmem_ld64(s_addr + 64, r);
+#pragma unroll
+        for (int u = 0; u < 64; ++u) s[64 + u] = __uint_as_float(r[u]);
+      }
+      const int key0 = j * C::BN;
+      const bool tail = key0 + C::BN > p.N;
+      const bool diag = p.causal && (key0 + C::BN - 1 > t_first);
+      if (tail || diag) {
+        const int lim = p.causal ? min(token, p.N - 1) : p.N - 1;  // last visible key
+#pragma unroll
+        for (int u = 0; u < 128; ++u)
+          if (key0 + u > lim) s[u] = -INFINITY;
+      }
+      float mx = s[0];
+#pragma unroll
+      for (int u = 1; u < 128; ++u) mx = fmaxf(mx, s[u]);
+      const float m_new = fmaxf(m, mx);
+      // Keep the stale maximum unless it grew by more than 2^8 in the exp2
+      // domain: O / l is exact either way, and P stays <= 256.
+      const bool need = (j == 0) || ((m_new - m) * sl2 > 8.0f);
+      const float m_use = need ? m_new : m;
+      const float f = (need && j > 0) ? ex2_approx((m - m_new) * sl2) : 1.0f;
+      const bool rescale = (j > 0) && __any_sync(0xffffffffu, need);
+      const float ms = m_use * sl2;
+      float lsum = 0.f;
+#pragma unroll
+      for (int u = 0; u < 128; ++u) {
+        s[u] = ex2_approx(fmaf(s[u], sl2, -ms));
+        lsum += s[u];
+      }
+      l = l * f + lsum;
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        uint32_t r[32];
+#pragma unroll
+        for (int u = 0; u < 32; ++u) r[u] = pack_bf16x2(s[c * 64 + 2 * u], s[c * 64 + 2 * u + 1]);
+        tmem_st32(s_addr + c * 32, r);
+      }
+      if (rescale) {
+        // O holds PV up to tile j-1 (complete: S_j was committed after it).
+#pragma unroll 1
+        for (int c = 0; c < D; c += 32) {
+          uint32_t r[32];
+          tmem_ld32(o_addr + c, r);
+#pragma unroll
+          for (int u = 0; u < 32; ++u) r[u] = __float_as_uint(__uint_as_float(r[u]) * f);
+          tmem_st32(o_addr + c, r);
+        }
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(C::BAR_P + k));
+      m = m_use;
+    }
+    if (ok && nk > 0 && mbar_wait_warp(bar(C::BAR_O + k), 0, ctl)) {
+      tc_fence_after();
+      const float inv_l = 1.0f / l;
+      const bool store = token < p.N;
+      __nv_bfloat16* dst = p.out + (((size_t)b * p.N + (store ? token : 0)) * p.H_q + head) * D;
+#pragma unroll
+      for (int c = 0; c < D; c += 32) {
+        uint32_t r[32];
+        tmem_ld32(o_addr + c, r);  // all lanes: the load is warp-collective
+        uint4 w[4];
+        uint32_t* wp = reinterpret_cast<uint32_t*>(w);
+#pragma unroll
+        for (int u = 0; u < 16; ++u)
+          wp[u] = pack_bf16x2(__uint_as_float(r[2 * u]) * inv_l, __uint_as_float(r[2 * u + 1]) * inv_l);
+        if (store) {
+          uint4* d4 = reinterpret_cast<uint4*>(dst + c);
+#pragma unroll
+          for (int u = 0; u < 4; ++u) d4[u] = w[u];
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 2) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+}  // namespace sqa

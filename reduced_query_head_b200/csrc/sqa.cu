@@ -1,0 +1,365 @@
+// libsqa C ABI: argument checks, TMA tensor maps, launches.
+// The declarations and their contracts are in include/sqa.h.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <climits>
+#include <cmath>
+#include <cstdint>
+#include <mutex>
+
+#include "sqa.h"
+#include "attn_fwd.cuh"
+#include "gemm.cuh"
+
+// Per-device status word written by kernels whose bounded waits ran out.
+__device__ int g_sqa_status;
+
+namespace {
+
+using sqa::AttnCfg;
+using sqa::AttnParams;
+using sqa::GemmCfg;
+using sqa::GemmParams;
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+constexpr int kMaxDevices = 64;
+constexpr unsigned long long kDefaultWaitNs = 2000000000ull;  // 2 s
+
+struct DeviceState {
+  bool ready = false;
+  int* status = nullptr;
+  int sms = 0;
+};
+
+std::mutex g_mu;
+DeviceState g_dev[kMaxDevices];
+EncodeTiledFn g_encode = nullptr;
+std::atomic<unsigned long long> g_wait_ns{kDefaultWaitNs};
+
+// One-time per-device set-up: status word address, SM count, shared-memory opt-in.
+int device_state(DeviceState** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return SQA_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_mu);
+  DeviceState& st = g_dev[dev];
+  if (!st.ready) {
+    if (!g_encode) {
+      void* fn = nullptr;
+      cudaDriverEntryPointQueryResult q;
+      if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000, cudaEnableDefault, &q) !=
+              cudaSuccess ||
+          q != cudaDriverEntryPointSuccess || !fn)
+        return SQA_ERR_CUDA;
+      g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+    }
+    if (cudaGetSymbolAddress(reinterpret_cast<void**>(&st.status), g_sqa_status) != cudaSuccess) return SQA_ERR_CUDA;
+    if (cudaDeviceGetAttribute(&st.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return SQA_ERR_CUDA;
+    if (cudaFuncSetAttribute(sqa::attn_fwd_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             AttnCfg<64>::SMEM_BYTES) != cudaSuccess ||
+        cudaFuncSetAttribute(sqa::attn_fwd_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             AttnCfg<128>::SMEM_BYTES) != cudaSuccess ||
+        cudaFuncSetAttribute(sqa::gemm_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             GemmCfg::SMEM_BYTES) != cudaSuccess)
+      return SQA_ERR_CUDA;
+    st.ready = true;
+  }
+  *out = &st;
+  return SQA_OK;
+}
+
+bool aligned16(const void* p) { return p != nullptr && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Tiled bf16 tensor map with 128-byte swizzle. dims/box innermost first;
+// strides in bytes for dims 1..rank-1.
+int encode_map(CUtensorMap* m, const void* base, int rank, const cuuint64_t* dims, const cuuint64_t* strides,
+               const cuuint32_t* box) {
+  const cuuint32_t es[5] = {1, 1, 1, 1, 1};
+  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void*>(base), dims, strides,
+                        box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? SQA_OK : SQA_ERR_CUDA;
+}
+
+int check_attn_args(const void* q, const void* k, const void* v, const void* out, int B, int N, int H_q, int H_kv,
+                    int d, int causal, float scale) {
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return SQA_ERR_INVALID_ARG;
+  if (B < 1 || N < 1 || H_q < 1 || H_kv < 1 || H_kv > H_q) return SQA_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return SQA_ERR_INVALID_ARG;
+  if (!(scale > 0.0f) || !std::isfinite(scale)) return SQA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return SQA_ERR_UNSUPPORTED;
+  // element counts must fit the 64-bit offsets; tensor-map strides < 2^40 bytes
+  const long double elems = (long double)B * N * H_q * d;
+  if (elems * 2 >= (long double)(1ull << 40)) return SQA_ERR_INVALID_ARG;
+  return SQA_OK;
+}
+
+// Heads stacked per 128-row tile: the largest power of two (<= 128) dividing
+// H_q / H_kv when the groups are even; otherwise one head per tile.
+int heads_per_tile(int H_q, int H_kv) {
+  if (H_q % H_kv != 0) return 1;
+  const int R = H_q / H_kv;
+  int P = 1;
+  while (P * 2 <= 128 && R % (P * 2) == 0) P *= 2;
+  return P;
+}
+
+template <int D>
+int launch_attn(const DeviceState* st, const void* q, const void* k, const void* v, void* out, int B, int N, int H_q,
+                int H_kv, int causal, float scale, cudaStream_t stream) {
+  using C = AttnCfg<D>;
+  const int P = heads_per_tile(H_q, H_kv);
+  int log2P = 0;
+  while ((1 << log2P) < P) ++log2P;
+  const int tpt = C::BM / P;
+  const long long n_pairs = ((long long)N + 2 * tpt - 1) / (2 * tpt);
+  const long long n_hb = H_q / P;
+  const long long grid = n_pairs * n_hb * B;
+  if (grid > INT_MAX) return SQA_ERR_INVALID_ARG;
+
+  CUtensorMap tq, tk, tv;
+  {
+    const cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)H_q, (cuuint64_t)N, (cuuint64_t)B};
+    const cuuint64_t strides[3] = {(cuuint64_t)D * 2, (cuuint64_t)H_q * D * 2, (cuuint64_t)N * H_q * D * 2};
+    const cuuint32_t box[4] = {64, (cuuint32_t)P, (cuuint32_t)tpt, 1};
+    if (int e = encode_map(&tq, q, 4, dims, strides, box)) return e;
+  }
+  {
+    const cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)H_kv, (cuuint64_t)N, (cuuint64_t)B};
+    const cuuint64_t strides[3] = {(cuuint64_t)D * 2, (cuuint64_t)H_kv * D * 2, (cuuint64_t)N * H_kv * D * 2};
+    const cuuint32_t box[4] = {64, 1, (cuuint32_t)C::BN, 1};
+    if (int e = encode_map(&tk, k, 4, dims, strides, box)) return e;
+    if (int e = encode_map(&tv, v, 4, dims, strides, box)) return e;
+  }
+  AttnParams p;
+  p.out = reinterpret_cast<__nv_bfloat16*>(out);
+  p.B = B;
+  p.N = N;
+  p.H_q = H_q;
+  p.H_kv = H_kv;
+  p.P = P;
+  p.log2P = log2P;
+  p.tpt = tpt;
+  p.n_pairs = (int)n_pairs;
+  p.n_hb = (int)n_hb;
+  p.causal = causal;
+  p.scale_log2 = (float)((double)scale * 1.4426950408889634);  // scale * log2(e)
+  p.status = st->status;
+  p.timeout_ns = g_wait_ns.load();
+  sqa::attn_fwd_kernel<D><<<(unsigned)grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);
+  return cudaGetLastError() == cudaSuccess ? SQA_OK : SQA_ERR_CUDA;
+}
+
+struct GemmOperands {
+  const void* x;
+  long long M;
+  int K;
+  int n_w;
+  const void* w[3];
+  int w_rows[3];
+  int N_out;
+  int n_y;
+  void* y[3];
+  int y_cols[3];  // width of each output (its row stride)
+};
+
+int launch_gemm(const DeviceState* st, const GemmOperands& g, cudaStream_t stream) {
+  using C = GemmCfg;
+  if (g.M > INT_MAX) return SQA_ERR_INVALID_ARG;
+  CUtensorMap tx, tw[3];
+  {
+    const cuuint64_t dims[2] = {(cuuint64_t)g.K, (cuuint64_t)g.M};
+    const cuuint64_t strides[1] = {(cuuint64_t)g.K * 2};
+    const cuuint32_t box[2] = {64, 128};
+    if (int e = encode_map(&tx, g.x, 2, dims, strides, box)) return e;
+  }
+  GemmParams p;
+  p.w_seg_start[0] = 0;
+  for (int i = 0; i < 3; ++i) {
+    const int idx = i < g.n_w ? i : 0;
+    const cuuint64_t dims[2] = {(cuuint64_t)g.K, (cuuint64_t)g.w_rows[idx]};
+    const cuuint64_t strides[1] = {(cuuint64_t)g.K * 2};
+    const cuuint32_t box[2] = {64, 64};
+    if (int e = encode_map(&tw[i], g.w[idx], 2, dims, strides, box)) return e;
+    if (i < g.n_w) p.w_seg_start[i + 1] = p.w_seg_start[i] + g.w_rows[i];
+  }
+  p.M = (int)g.M;
+  p.K = g.K;
+  p.N_out = g.N_out;
+  p.tiles_m = (int)((g.M + C::BM - 1) / C::BM);
+  p.tiles_n = (g.N_out + C::BN - 1) / C::BN;
+  p.n_seg_w = g.n_w;
+  p.n_seg_y = g.n_y;
+  p.y_seg_start[0] = 0;
+  for (int i = 0; i < 3; ++i) {
+    p.y_ptr[i] = reinterpret_cast<__nv_bfloat16*>(i < g.n_y ? g.y[i] : g.y[0]);
+    p.y_ld[i] = i < g.n_y ? g.y_cols[i] : g.y_cols[0];
+    if (i < g.n_y) p.y_seg_start[i + 1] = p.y_seg_start[i] + g.y_cols[i];
+  }
+  p.status = st->status;
+  p.timeout_ns = g_wait_ns.load();
+  const long long tiles = (long long)p.tiles_m * p.tiles_n;
+  if (tiles > INT_MAX) return SQA_ERR_INVALID_ARG;
+  const int grid = (int)(tiles < st->sms ? tiles : st->sms);
+  sqa::gemm_bf16_kernel<<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tx, tw[0], tw[1], tw[2], p);
+  return cudaGetLastError() == cudaSuccess ? SQA_OK : SQA_ERR_CUDA;
+}
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+__global__ void wait_probe_kernel(int* status, unsigned long long ns) {
+  __shared__ alignas(8) uint64_t barrier;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    sqa::mbar_init(sqa::smem_u32(&barrier), 1);
+    abort_flag = 0;
+    sqa::fence_mbar_init();
+  }
+  __syncthreads();
+  sqa::WaitCtl c{&abort_flag, status, ns};
+  sqa::mbar_wait_warp(sqa::smem_u32(&barrier), 0, c);  // nothing arrives: must give up
+}
+
+}  // namespace
+
+extern "C" {
+
+int sqa_attn_fwd(const void* q, const void* k, const void* v, void* out, int B, int N, int H_q, int H_kv, int d_head,
+                 int causal, float scale, void* stream) {
+  if (int e = check_attn_args(q, k, v, out, B, N, H_q, H_kv, d_head, causal, scale)) return e;
+  DeviceState* st = nullptr;
+  if (int e = device_state(&st)) return e;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  return d_head == 64 ? launch_attn<64>(st, q, k, v, out, B, N, H_q, H_kv, causal, scale, s)
+                      : launch_attn<128>(st, q, k, v, out, B, N, H_q, H_kv, causal, scale, s);
+}
+
+size_t sqa_layer_workspace_bytes(int B, int N, int d_model, int H_q, int H_kv, int d_head) {
+  if (B < 1 || N < 1 || d_model < 8 || H_q < 1 || H_kv < 1 || H_kv > H_q || d_head < 1) return 0;
+  const size_t M = (size_t)B * N;
+  return align256(M * H_q * d_head * 2) * 2 + align256(M * H_kv * d_head * 2) * 2;
+}
+
+int sqa_layer_fwd(const void* x, const void* Wq, const void* Wk, const void* Wv, const void* Wo, void* out,
+                  void* workspace, size_t workspace_bytes, int B, int N, int d_model, int H_q, int H_kv, int d_head,
+                  int causal, float scale, void* stream) {
+  if (!aligned16(x) || !aligned16(Wq) || !aligned16(Wk) || !aligned16(Wv) || !aligned16(Wo) || !aligned16(out))
+    return SQA_ERR_INVALID_ARG;
+  if (d_model < 8 || d_model % 8 != 0) return SQA_ERR_INVALID_ARG;
+  if (B < 1 || N < 1 || H_q < 1 || H_kv < 1 || H_kv > H_q) return SQA_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return SQA_ERR_INVALID_ARG;
+  if (!(scale > 0.0f) || !std::isfinite(scale)) return SQA_ERR_INVALID_ARG;
+  if (d_head != 64 && d_head != 128) return SQA_ERR_UNSUPPORTED;
+  const long long M = (long long)B * N;
+  if (M > INT_MAX || (long double)M * d_model * 2 >= (long double)(1ull << 40)) return SQA_ERR_INVALID_ARG;
+  const size_t need = sqa_layer_workspace_bytes(B, N, d_model, H_q, H_kv, d_head);
+  if (workspace == nullptr || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 || workspace_bytes < need)
+    return SQA_ERR_WORKSPACE;
+  DeviceState* st = nullptr;
+  if (int e = device_state(&st)) return e;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+
+  uint8_t* ws = reinterpret_cast<uint8_t*>(workspace);
+  const size_t q_bytes = align256((size_t)M * H_q * d_head * 2);
+  const size_t kv_bytes = align256((size_t)M * H_kv * d_head * 2);
+  void* Q = ws;
+  void* K = ws + q_bytes;
+  void* V = ws + q_bytes + kv_bytes;
+  void* A = ws + q_bytes + 2 * kv_bytes;
+
+  GemmOperands g1{};
+  g1.x = x;
+  g1.M = M;
+  g1.K = d_model;
+  g1.n_w = 3;
+  g1.w[0] = Wq; g1.w[1] = Wk; g1.w[2] = Wv;
+  g1.w_rows[0] = H_q * d_head; g1.w_rows[1] = H_kv * d_head; g1.w_rows[2] = H_kv * d_head;
+  g1.N_out = (H_q + 2 * H_kv) * d_head;
+  g1.n_y = 3;
+  g1.y[0] = Q; g1.y[1] = K; g1.y[2] = V;
+  g1.y_cols[0] = H_q * d_head; g1.y_cols[1] = H_kv * d_head; g1.y_cols[2] = H_kv * d_head;
+  if (int e = launch_gemm(st, g1, s)) return e;
+
+  if (int e = d_head == 64 ? launch_attn<64>(st, Q, K, V, A, B, N, H_q, H_kv, causal, scale, s)
+                           : launch_attn<128>(st, Q, K, V, A, B, N, H_q, H_kv, causal, scale, s))
+    return e;
+
+  GemmOperands g2{};
+  g2.x = A;
+  g2.M = M;
+  g2.K = H_q * d_head;
+  g2.n_w = 1;
+  g2.w[0] = Wo;
+  g2.w_rows[0] = d_model;
+  g2.N_out = d_model;
+  g2.n_y = 1;
+  g2.y[0] = out;
+  g2.y_cols[0] = d_model;
+  return launch_gemm(st, g2, s);
+}
+
+int sqa_linear_fwd(const void* x, const void* W, void* y, long long M, int K, int N_out, void* stream) {
+  if (!aligned16(x) || !aligned16(W) || !aligned16(y)) return SQA_ERR_INVALID_ARG;
+  if (M < 1 || M > INT_MAX || K < 8 || K % 8 != 0 || N_out < 8 || N_out % 8 != 0) return SQA_ERR_INVALID_ARG;
+  if ((long double)M * K * 2 >= (long double)(1ull << 40) || (long double)N_out * K * 2 >= (long double)(1ull << 40))
+    return SQA_ERR_INVALID_ARG;
+  DeviceState* st = nullptr;
+  if (int e = device_state(&st)) return e;
+  GemmOperands g{};
+  g.x = x;
+  g.M = M;
+  g.K = K;
+  g.n_w = 1;
+  g.w[0] = W;
+  g.w_rows[0] = N_out;
+  g.N_out = N_out;
+  g.n_y = 1;
+  g.y[0] = y;
+  g.y_cols[0] = N_out;
+  return launch_gemm(st, g, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int sqa_device_status(void* stream) {
+  DeviceState* st = nullptr;
+  if (int e = device_state(&st)) return e;
+  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return SQA_ERR_CUDA;
+  int v = 0;
+  const int zero = 0;
+  if (cudaMemcpyFromSymbol(&v, g_sqa_status, sizeof v) != cudaSuccess) return SQA_ERR_CUDA;
+  if (cudaMemcpyToSymbol(g_sqa_status, &zero, sizeof zero) != cudaSuccess) return SQA_ERR_CUDA;
+  return v;
+}
+
+unsigned long long sqa_set_wait_limit_ns(unsigned long long ns) {
+  return g_wait_ns.exchange(ns == 0 ? kDefaultWaitNs : ns);
+}
+
+int sqa_check_wait_timeout(unsigned long long limit_ns, void* stream) {
+  if (limit_ns < 1000ull || limit_ns > 10000000000ull) return SQA_ERR_INVALID_ARG;
+  DeviceState* st = nullptr;
+  if (int e = device_state(&st)) return e;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  wait_probe_kernel<<<1, 32, 0, s>>>(st->status, limit_ns);
+  if (cudaGetLastError() != cudaSuccess) return SQA_ERR_CUDA;
+  return sqa_device_status(stream);
+}
+
+const char* sqa_status_string(int status) {
+  switch (status) {
+    case SQA_OK: return "SQA_OK";
+    case SQA_ERR_INVALID_ARG: return "SQA_ERR_INVALID_ARG";
+    case SQA_ERR_UNSUPPORTED: return "SQA_ERR_UNSUPPORTED";
+    case SQA_ERR_CUDA: return "SQA_ERR_CUDA";
+    case SQA_ERR_TIMEOUT: return "SQA_ERR_TIMEOUT";
+    case SQA_ERR_WORKSPACE: return "SQA_ERR_WORKSPACE";
+    default: return "SQA_ERR_UNKNOWN";
+  }
+}
+
+int sqa_version(void) { return 100; }
+
+}  // extern "C"

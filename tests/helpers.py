@@ -1,0 +1,98 @@
+"""Shared helpers for the parity tests: seeded inputs, error metrics, configs."""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+import synth
+
+# Acceptance bar for bf16-in / fp32-accumulate attention against the float64
+# oracle: max-abs error and relative L2 error over the compared outputs.
+MAX_ABS_TOL = 1e-2
+REL_L2_TOL = 5e-3
+N_SAMPLED_ROWS = 1024
+
+
+def errors(got: np.ndarray, want: np.ndarray):
+    got = np.asarray(got, dtype=np.float64)
+    want = np.asarray(want, dtype=np.float64)
+    diff = got - want
+    max_abs = float(np.max(np.abs(diff))) if diff.size else 0.0
+    den = float(np.linalg.norm(want.ravel()))
+    rel = float(np.linalg.norm(diff.ravel()) / den) if den > 0 else float(np.linalg.norm(diff.ravel()))
+    return max_abs, rel
+
+
+def assert_close(got, want, what=""):
+    max_abs, rel = errors(got, want)
+    assert np.all(np.isfinite(got)), "%s: non-finite output" % what
+    assert max_abs <= MAX_ABS_TOL and rel <= REL_L2_TOL, \
+        "%s: max_abs=%.3e (tol %.0e) rel_l2=%.3e (tol %.0e)" % (what, max_abs, MAX_ABS_TOL, rel, REL_L2_TOL)
+    return max_abs, rel
+
+
+def attn_inputs(B, N, H_q, H_kv, d, seed=0, factor=1.0):
+    """bf16 bit arrays q [B,N,H_q,d], k/v [B,N,H_kv,d] from the seeded generator."""
+    q = synth.bf16_bits((B, N, H_q, d), seed, "q", factor)
+    k = synth.bf16_bits((B, N, H_kv, d), seed, "k", factor)
+    v = synth.bf16_bits((B, N, H_kv, d), seed, "v", factor)
+    return q, k, v
+
+
+def sampled_rows(B, N, seed, n=N_SAMPLED_ROWS):
+    """>= n seeded flat positions b*N+t, always including the tile edges."""
+    must = [0, N - 1, 127, 128]
+    if N % 128:
+        must.append(N - 1 - (N % 128))
+    extra = []
+    for b in range(B):
+        extra += [b * N + t for t in must]
+    return synth.sample_rows(n, B * N, seed ^ 0x5A17, must_include=extra)
+
+
+# Config 5 grid: N x H_q x H_kv (H_kv <= H_q), row-major in the listed order;
+# the position in this list is the seed.
+def cost_sweep_grid():
+    grid = []
+    for N in (32768, 65536, 131072, 200000):
+        for H_q in (32, 16, 8, 4):
+            for H_kv in (8, 4, 1):
+                if H_kv <= H_q:
+                    grid.append((N, H_q, H_kv))
+    return grid
+
+
+HEAD_CONFIGS_32K = [("MHA", 16, 16), ("GQA", 16, 4), ("MQA", 16, 1), ("SQA", 8, 4), ("sSQA", 8, 8),
+                    ("xSQA", 4, 4), ("xSMQA", 4, 1)]
+LONG_HEAD_CONFIGS = [("MHA", 16, 16), ("SQA", 8, 4), ("xSQA", 4, 4)]
+
+
+def default_scale(d):
+    return 1.0 / math.sqrt(d)
+
+
+# ---------------------------------------------------------------- GPU side
+def to_device_bf16(bits: np.ndarray):
+    import torch
+    t = torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16)
+    return t.cuda()
+
+
+def bf16_tensor_to_f64(t) -> np.ndarray:
+    import torch
+    return t.detach().to(torch.float32).cpu().numpy().astype(np.float64)
+
+
+def run_attn(q_bits, k_bits, v_bits, causal, scale, d=None):
+    """Run sqa_attn_fwd through the C ABI on device copies of the bit arrays."""
+    import torch
+    import reduced_query_head_b200 as sqa
+    B, N, H_q, dd = q_bits.shape
+    H_kv = k_bits.shape[2]
+    q, k, v = to_device_bf16(q_bits), to_device_bf16(k_bits), to_device_bf16(v_bits)
+    out = torch.full((B, N, H_q, dd), float("nan"), dtype=torch.bfloat16, device="cuda")
+    sqa.sqa_attn_fwd(q, k, v, out, B, N, H_q, H_kv, dd, int(causal), scale)
+    st = sqa.sqa_device_status()
+    assert st == sqa.SQA_OK, sqa.sqa_status_string(st)
+    return out

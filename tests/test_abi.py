@@ -1,0 +1,111 @@
+"""The C-ABI library loads and exports every declared symbol; host-side checks.
+
+Runs without a GPU: only entry points that return before touching the device
+are called (argument validation, status strings, sizes).
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_functions():
+    with open(os.path.join(ROOT, "include", "sqa.h")) as f:
+        text = f.read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(sqa_[a-z0-9_]+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def sqa():
+    from reduced_query_head_b200 import build
+    build.build()
+    import reduced_query_head_b200
+    return reduced_query_head_b200
+
+
+def test_header_declares_the_boundary():
+    fns = _declared_functions()
+    for name in ("sqa_attn_fwd", "sqa_layer_fwd", "sqa_layer_workspace_bytes", "sqa_device_status",
+                 "sqa_status_string"):
+        assert name in fns
+
+
+def test_library_exports_every_declared_symbol(sqa):
+    lib = ctypes.CDLL(sqa.build.LIB)
+    for name in _declared_functions():
+        assert hasattr(lib, name), name
+    assert set(_declared_functions()) == set(sqa.EXPORTED_SYMBOLS)
+
+
+def test_status_strings_and_version(sqa):
+    assert sqa.sqa_status_string(sqa.SQA_OK) == "SQA_OK"
+    assert sqa.sqa_status_string(sqa.SQA_ERR_TIMEOUT) == "SQA_ERR_TIMEOUT"
+    assert sqa.sqa_status_string(99) == "SQA_ERR_UNKNOWN"
+    assert sqa.sqa_version() >= 100
+
+
+P = 1 << 20  # a 16-byte aligned fake address; never dereferenced (validation fails first)
+
+
+@pytest.mark.parametrize("args,code", [
+    ((0, P, P, P, 1, 128, 8, 4, 64, 0, 0.125), 1),        # null q
+    ((P + 2, P, P, P, 1, 128, 8, 4, 64, 0, 0.125), 1),    # misaligned q
+    ((P, P, P, P, 0, 128, 8, 4, 64, 0, 0.125), 1),        # B = 0
+    ((P, P, P, P, 1, 0, 8, 4, 64, 0, 0.125), 1),          # N = 0
+    ((P, P, P, P, 1, 128, 4, 8, 64, 0, 0.125), 1),        # H_kv > H_q
+    ((P, P, P, P, 1, 128, 8, 0, 64, 0, 0.125), 1),        # H_kv = 0
+    ((P, P, P, P, 1, 128, 8, 4, 64, 2, 0.125), 1),        # causal not 0/1
+    ((P, P, P, P, 1, 128, 8, 4, 64, 0, 0.0), 1),          # scale 0
+    ((P, P, P, P, 1, 128, 8, 4, 64, 0, -1.0), 1),         # negative scale
+    ((P, P, P, P, 1, 128, 8, 4, 64, 0, float("nan")), 1),
+    ((P, P, P, P, 1, 128, 8, 4, 64, 0, float("inf")), 1),
+    ((P, P, P, P, 1, 128, 8, 4, 96, 0, 0.125), 2),        # d_head unsupported
+    ((P, P, P, P, 1, 128, 8, 4, 32, 0, 0.125), 2),
+    ((P, P, P, P, 1 << 16, 1 << 16, 64, 8, 128, 0, 0.1), 1),  # too large for 40-bit strides
+])
+def test_attn_argument_validation(sqa, args, code):
+    st = sqa.lib.sqa_attn_fwd(*args[:10], ctypes.c_float(args[10]), None)
+    assert st == code, sqa.sqa_status_string(st)
+
+
+def test_layer_workspace_size(sqa):
+    B, N, dm, H_q, H_kv, d = 4, 16384, 2048, 16, 8, 64
+    M = B * N
+    want = 2 * M * H_q * d * 2 + 2 * M * H_kv * d * 2
+    assert sqa.sqa_layer_workspace_bytes(B, N, dm, H_q, H_kv, d) == want
+    assert sqa.sqa_layer_workspace_bytes(1, 3, 16, 2, 1, 64) % 256 == 0
+    assert sqa.sqa_layer_workspace_bytes(0, 3, 16, 2, 1, 64) == 0
+    assert sqa.sqa_layer_workspace_bytes(1, 3, 16, 1, 2, 64) == 0
+
+
+def test_layer_argument_validation(sqa):
+    L = sqa.lib
+    ws = sqa.sqa_layer_workspace_bytes(1, 128, 64, 2, 1, 64)
+    ok = (P, P, P, P, P, P, P, ws, 1, 128, 64, 2, 1, 64, 1)
+    assert L.sqa_layer_fwd(*ok[:7], ws - 256, *ok[8:], ctypes.c_float(0.125), None) == 5   # small workspace
+    assert L.sqa_layer_fwd(*ok[:6], P + 16, *ok[7:], ctypes.c_float(0.125), None) == 5     # misaligned ws
+    assert L.sqa_layer_fwd(*ok[:6], 0, *ok[7:], ctypes.c_float(0.125), None) == 5          # null ws
+    bad_dm = ok[:10] + (60,) + ok[11:]
+    assert L.sqa_layer_fwd(*bad_dm, ctypes.c_float(0.125), None) == 1                      # d_model % 8
+    bad_d = ok[:13] + (80,) + ok[14:]
+    assert L.sqa_layer_fwd(*bad_d, ctypes.c_float(0.125), None) == 2
+    assert L.sqa_layer_fwd(0, *ok[1:], ctypes.c_float(0.125), None) == 1                   # null x
+
+
+def test_linear_argument_validation(sqa):
+    L = sqa.lib
+    assert L.sqa_linear_fwd(P, P, P, 0, 64, 64, None) == 1
+    assert L.sqa_linear_fwd(P, P, P, 16, 60, 64, None) == 1
+    assert L.sqa_linear_fwd(P, P, P, 16, 64, 36, None) == 1
+    assert L.sqa_linear_fwd(P, 0, P, 16, 64, 64, None) == 1
+
+
+def test_wait_limit_roundtrip(sqa):
+    prev = sqa.sqa_set_wait_limit_ns(12345)
+    assert sqa.sqa_set_wait_limit_ns(0) == 12345
+    assert sqa.sqa_set_wait_limit_ns(prev) == 2_000_000_000
+    assert sqa.lib.sqa_check_wait_timeout(10, None) == 1      # limit below range -> invalid

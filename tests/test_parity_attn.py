@@ -1,0 +1,114 @@
+"""GPU parity: sqa_attn_fwd (CUDA, through the C ABI) against the float64 oracle.
+
+Same seeded bf16 inputs on both sides. Small shapes compare every output
+element; the long-sequence configurations compare >= 1024 seeded query
+positions (all heads each), always including the first/last token and the
+tile edges. Bar: max-abs <= 1e-2 and relative L2 <= 5e-3 (bf16 in, fp32
+accumulate, against float64).
+"""
+import numpy as np
+import pytest
+
+import oracle
+from helpers import (HEAD_CONFIGS_32K, LONG_HEAD_CONFIGS, assert_close, attn_inputs, bf16_tensor_to_f64,
+                     cost_sweep_grid, default_scale, run_attn, sampled_rows)
+
+pytestmark = pytest.mark.gpu
+
+
+def _full_check(B, N, H_q, H_kv, d, causal, scale=None, seed=0, factor=1.0, what=""):
+    scale = default_scale(d) if scale is None else scale
+    qb, kb, vb = attn_inputs(B, N, H_q, H_kv, d, seed, factor)
+    out = bf16_tensor_to_f64(run_attn(qb, kb, vb, causal, scale))
+    want = oracle.attention(oracle.widen_bf16(qb), oracle.widen_bf16(kb), oracle.widen_bf16(vb), causal, scale)
+    return assert_close(out, want, what or str((B, N, H_q, H_kv, d, causal)))
+
+
+def _sampled_check(B, N, H_q, H_kv, d, causal, seed, factor=1.0, scale=None, what=""):
+    import torch
+    scale = default_scale(d) if scale is None else scale
+    qb, kb, vb = attn_inputs(B, N, H_q, H_kv, d, seed, factor)
+    out = run_attn(qb, kb, vb, causal, scale)
+    rows = sampled_rows(B, N, seed)
+    got = bf16_tensor_to_f64(out.view(B * N, H_q, d)[torch.from_numpy(rows).cuda()])
+    del out
+    q_rows = oracle.widen_bf16(qb.reshape(B * N, H_q, d)[rows])
+    want = oracle.attention_rows(q_rows, oracle.widen_bf16(kb), oracle.widen_bf16(vb), rows, N, causal, scale)
+    return assert_close(got, want, what or str((B, N, H_q, H_kv, d, causal)))
+
+
+# ------------------------------------------------------------ config 1 (full output)
+def test_config1_small_sqa_full_output():
+    """B=1, N=1024, H_q=8, H_kv=4, d=64, non-causal, scale 1/8, seed 0."""
+    _full_check(1, 1024, 8, 4, 64, False, 1.0 / 8.0, seed=0)
+
+
+# ------------------------------------------------------------ edge shapes (full output)
+EDGE = [
+    # B, N, H_q, H_kv, d
+    (1, 1, 1, 1, 64),        # one token
+    (1, 2, 2, 1, 64),
+    (1, 127, 4, 4, 64),      # ragged tile
+    (1, 128, 8, 2, 64),      # exactly one tile
+    (1, 129, 16, 1, 64),     # one past a tile, MQA, 16 heads stacked
+    (2, 255, 4, 2, 128),     # batch 2, d=128
+    (1, 1000, 8, 4, 128),
+    (3, 300, 6, 4, 64),      # uneven groups: floor map, one head per tile
+    (1, 257, 32, 1, 64),     # 32 heads stacked per tile
+    (1, 513, 12, 3, 128),    # R=4 with 12 heads
+    (2, 700, 5, 5, 64),      # MHA with odd head count
+    (1, 384, 3, 1, 128),     # R=3, one head per tile
+    (1, 1025, 64, 2, 64),    # R=32
+    (1, 640, 128, 1, 64),    # R=128: one token per tile
+]
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("shape", EDGE, ids=lambda s: "B%dN%dHq%dHkv%dd%d" % s)
+def test_edge_shapes_full_output(shape, causal):
+    _full_check(*shape, causal, seed=11)
+
+
+@pytest.mark.parametrize("scale", [0.02, 0.3, 1.0])
+def test_nondefault_scale(scale):
+    _full_check(1, 300, 4, 2, 64, True, scale=scale, seed=3)
+    _full_check(1, 300, 4, 2, 128, False, scale=scale, seed=4)
+
+
+def test_large_scores_stress_rescale():
+    # values x4 make score rows peaky, so the running max moves by > 2^8 often
+    _full_check(1, 2048, 4, 1, 64, False, seed=5, factor=2.0)
+    _full_check(1, 2048, 4, 1, 128, True, seed=6, factor=2.0)
+
+
+def test_deterministic_bitwise():
+    qb, kb, vb = attn_inputs(1, 3000, 8, 2, 64, 21)
+    a = run_attn(qb, kb, vb, True, 0.125)
+    b = run_attn(qb, kb, vb, True, 0.125)
+    assert bool((a.view(-1).view(dtype=__import__("torch").int16) ==
+                 b.view(-1).view(dtype=__import__("torch").int16)).all())
+
+
+# ------------------------------------------------------------ config 2 (sampled rows)
+@pytest.mark.parametrize("name,H_q,H_kv", HEAD_CONFIGS_32K, ids=[c[0] for c in HEAD_CONFIGS_32K])
+def test_config2_head_configs_32k(name, H_q, H_kv):
+    _sampled_check(1, 32768, H_q, H_kv, 64, False, seed=0, what="config2 " + name)
+
+
+# ------------------------------------------------------------ config 3 (sampled rows)
+@pytest.mark.parametrize("N", [65536, 131072, 200000])
+@pytest.mark.parametrize("name,H_q,H_kv", LONG_HEAD_CONFIGS, ids=[c[0] for c in LONG_HEAD_CONFIGS])
+def test_config3_long_sequences(name, H_q, H_kv, N):
+    _sampled_check(1, N, H_q, H_kv, 64, False, seed=0, what="config3 %s N=%d" % (name, N))
+
+
+# ------------------------------------------------------------ config 5 (sampled rows)
+GRID = cost_sweep_grid()
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("idx", range(len(GRID)), ids=["N%dHq%dHkv%d" % g for g in GRID])
+def test_config5_cost_sweep(idx, causal):
+    N, H_q, H_kv = GRID[idx]
+    _sampled_check(1, N, H_q, H_kv, 128, causal, seed=idx, factor=0.5,
+                   what="config5 #%d N=%d Hq=%d Hkv=%d causal=%d" % (idx, N, H_q, H_kv, causal))
