@@ -397,6 +397,23 @@ def bench_extra(args):
                           "pct_of_peak": round(100 * fl / (med * 1e-3) / 1e12 / peaks["bf16_tflops"], 1)})
             print(json.dumps(lines[-1]), flush=True)
             del dev, out
+    elif args.workload == "single":
+        # one attention configuration, e.g. for a profiler capture
+        N, H_q, H_kv, d, causal = args.N, args.hq, args.hkv, args.d, args.causal
+        _, dev = make_attn_inputs(1, N, H_q, H_kv, d, 0, 1.0, device)
+        out = torch.empty((1, N, H_q, d), dtype=torch.bfloat16, device=device)
+
+        def fn():
+            sqa.sqa_attn_fwd(dev["q"], dev["k"], dev["v"], out, 1, N, H_q, H_kv, d, causal, d ** -0.5, stream)
+        for _ in range(args.warmup):
+            fn()
+        ms = _time_launches(fn, args.steps, flush, stream)
+        assert sqa.sqa_device_status(stream) == 0
+        fl = attn_flops(1, N, H_q, d, causal)
+        med = statistics.median(ms)
+        lines.append({"workload": "single", "N": N, "H_q": H_q, "H_kv": H_kv, "d": d, "causal": causal,
+                      "ms_median": round(med, 3), "tflops": round(fl / (med * 1e-3) / 1e12, 1)})
+        print(json.dumps(lines[-1]), flush=True)
     elif args.workload == "layer":
         import synth
         B, N, dm, H_q, H_kv, d = 4, 16384, 2048, 16, 8, 64
@@ -447,13 +464,18 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["sqa", "reference"], default="sqa")
-    ap.add_argument("--workload", choices=["headcfg32k", "long", "layer", "sweep"], default="headcfg32k")
+    ap.add_argument("--workload", choices=["headcfg32k", "long", "layer", "sweep", "single"], default="headcfg32k")
+    ap.add_argument("--N", type=int, default=32768)
+    ap.add_argument("--hq", type=int, default=16)
+    ap.add_argument("--hkv", type=int, default=16)
+    ap.add_argument("--d", type=int, default=64)
+    ap.add_argument("--causal", type=int, default=0)
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--traffic", type=float, default=None,
                     help="ncu dram bytes per attention launch, if captured for this kernel build")
     args = ap.parse_args()
-    if args.warmup < 3 and args.impl == "sqa":
+    if args.warmup < 3 and args.impl == "sqa" and args.workload == "headcfg32k":
         print("note: raising --warmup to 3", file=sys.stderr)
         args.warmup = 3
     if args.impl == "reference":

@@ -24,11 +24,27 @@ def errors(got: np.ndarray, want: np.ndarray):
     return max_abs, rel
 
 
-def assert_close(got, want, what=""):
+# Outside the five stated configurations (edge shapes, other scales, plain
+# GEMMs) outputs can exceed 2 in magnitude, where one bf16 rounding step of the
+# output alone is up to 2^-8 |y| (0.0156 at |y| = 4). There the per-element
+# bound adds that rounding term: |got - want| <= 1e-2 + 2^-8 |want|.
+BF16_OUT_REL = 2.0 ** -8
+
+
+def assert_close(got, want, what="", out_rounding=False):
+    got = np.asarray(got, dtype=np.float64)
+    want = np.asarray(want, dtype=np.float64)
     max_abs, rel = errors(got, want)
     assert np.all(np.isfinite(got)), "%s: non-finite output" % what
-    assert max_abs <= MAX_ABS_TOL and rel <= REL_L2_TOL, \
-        "%s: max_abs=%.3e (tol %.0e) rel_l2=%.3e (tol %.0e)" % (what, max_abs, MAX_ABS_TOL, rel, REL_L2_TOL)
+    if out_rounding:
+        excess = np.abs(got - want) - (MAX_ABS_TOL + BF16_OUT_REL * np.abs(want))
+        worst = float(excess.max()) if excess.size else 0.0
+        assert worst <= 0 and rel <= REL_L2_TOL, \
+            "%s: max_abs=%.3e exceeds 1e-2 + 2^-8|want| by %.3e; rel_l2=%.3e (tol %.0e)" % (
+                what, max_abs, worst, rel, REL_L2_TOL)
+    else:
+        assert max_abs <= MAX_ABS_TOL and rel <= REL_L2_TOL, \
+            "%s: max_abs=%.3e (tol %.0e) rel_l2=%.3e (tol %.0e)" % (what, max_abs, MAX_ABS_TOL, rel, REL_L2_TOL)
     return max_abs, rel
 
 

@@ -29,7 +29,7 @@ def _linear(M, K, N_out, seed):
                                        (1000, 512, 520), (129, 1024, 768), (4096, 2048, 2048)])
 def test_linear_matches_float64(M, K, N_out):
     got, want = _linear(M, K, N_out, 7)
-    assert_close(got, want, "linear %dx%dx%d" % (M, K, N_out))
+    assert_close(got, want, "linear %dx%dx%d" % (M, K, N_out), out_rounding=True)
 
 
 def _layer_inputs(B, N, dm, H_q, H_kv, d, seed):
@@ -65,7 +65,7 @@ def test_layer_small_full(B, N, dm, H_q, H_kv, d, causal):
     got = bf16_tensor_to_f64(_run_layer(bits, B, N, dm, H_q, H_kv, d, causal, scale))
     f = [oracle.widen_bf16(b) for b in bits]
     want = oracle.layer(f[0], f[1], f[2], f[3], f[4], H_q, H_kv, d, causal, scale, storage_rounding=True)
-    assert_close(got, want, "layer")
+    assert_close(got, want, "layer", out_rounding=True)
     # the pure float64 chain differs only by the bf16 storage rounding
     want64 = oracle.layer(f[0], f[1], f[2], f[3], f[4], H_q, H_kv, d, causal, scale, storage_rounding=False)
     assert errors(got, want64)[1] < 2e-2
