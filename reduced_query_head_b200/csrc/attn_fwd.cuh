@@ -52,29 +52,41 @@ struct AttnCfg {
   static constexpr int KV_BYTES = BN * D * 2;           // one K (or V) tile
   static constexpr int CHUNK_Q = BM * 128;              // bytes per column chunk
   static constexpr int CHUNK_KV = BN * 128;
+  // P gets its own TMEM columns when they fit (d = 64); at d = 128 it is
+  // written over the first half of S.
+  static constexpr bool SEP_P = (D == 64);
   // shared-memory map (offsets from a 1024-aligned base)
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + 2 * Q_BYTES;
   static constexpr int OFF_V = OFF_K + STAGES * KV_BYTES;
   static constexpr int OFF_BAR = OFF_V + STAGES * KV_BYTES;
-  // barriers: q_full, k_full[S], v_full[S], kv_empty[S], s_full[2], p_full[2], o_full[2], drain
+  // barriers
   static constexpr int BAR_Q = 0;
-  static constexpr int BAR_KF = 1;
-  static constexpr int BAR_VF = BAR_KF + STAGES;
-  static constexpr int BAR_KVE = BAR_VF + STAGES;
-  static constexpr int BAR_S = BAR_KVE + STAGES;
-  static constexpr int BAR_P = BAR_S + 2;
-  static constexpr int BAR_O = BAR_P + 2;
+  static constexpr int BAR_KF = 1;                      // [STAGES] K tile landed
+  static constexpr int BAR_VF = BAR_KF + STAGES;        // [STAGES] V tile landed
+  static constexpr int BAR_KVE = BAR_VF + STAGES;       // [STAGES] stage free again
+  static constexpr int BAR_S = BAR_KVE + STAGES;        // [2] S_k ready in TMEM
+  static constexpr int BAR_SFREE = BAR_S + 2;           // [2] S_k read out by softmax (4 warps)
+  static constexpr int BAR_P = BAR_SFREE + 2;           // [2] P_k written, O_k corrected (4 warps)
+  static constexpr int BAR_PV = BAR_P + 2;              // [2] O_k += P_k V done
+  static constexpr int BAR_O = BAR_PV + 2;              // [2] last PV of tile k done
   static constexpr int BAR_DRAIN = BAR_O + 2;
   static constexpr int N_BARS = BAR_DRAIN + 1;
   static constexpr int OFF_MISC = OFF_BAR + N_BARS * 8;  // tmem base (u32), abort flag (u32)
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;  // + alignment slack
   static constexpr int THREADS = 384;
+  static constexpr int REGS_LAUNCH = 168, REGS_CTRL = 56, REGS_SOFTMAX = 224;
   static constexpr uint32_t TMEM_COLS = 512;
-  static constexpr uint32_t COL_S0 = 0, COL_S1 = 128, COL_O0 = 256, COL_O1 = 256 + D;
+  static constexpr uint32_t COL_S0 = 0, COL_S1 = 128;
+  static constexpr uint32_t COL_O0 = 256, COL_O1 = 256 + D;
+  static constexpr uint32_t COL_P0 = SEP_P ? 256 + 2 * D : COL_S0;
+  static constexpr uint32_t COL_P1 = SEP_P ? 256 + 2 * D + 64 : COL_S1;
+  static_assert(!SEP_P || COL_P1 + 64 <= TMEM_COLS, "TMEM budget");
 };
 
-template <int D>
+// EMU: of every 8 column pairs of a score row, how many take 2^x from the
+// polynomial on the FMA pipe instead of the MUFU unit (0..8).
+template <int D, int EMU>
 __global__ void __launch_bounds__(384, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
@@ -120,7 +132,10 @@ __global__ void __launch_bounds__(384, 1)
   WaitCtl ctl{abort_flag, p.status, p.timeout_ns};
 
   if (tid == 0) {
-    for (int i = 0; i < C::N_BARS; ++i) mbar_init(bar(i), (i == C::BAR_P || i == C::BAR_P + 1) ? 4 : 1);
+    for (int i = 0; i < C::N_BARS; ++i) {
+      const bool per_warp = (i >= C::BAR_SFREE && i < C::BAR_SFREE + 2) || (i >= C::BAR_P && i < C::BAR_P + 2);
+      mbar_init(bar(i), per_warp ? 4 : 1);
+    }
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -132,6 +147,13 @@ __global__ void __launch_bounds__(384, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+
+  // Register split: the kernel launches with REGS_LAUNCH per thread (the host
+  // checks this before launching). Warpgroup 0 (producer, MMA, TMEM owner)
+  // gives registers back, the two softmax warpgroups take them:
+  // 128*REGS_CTRL + 256*REGS_SOFTMAX == 384*REGS_LAUNCH.
+  static_assert(128 * C::REGS_CTRL + 256 * C::REGS_SOFTMAX == 384 * C::REGS_LAUNCH, "register split");
+  if (warp < 4) regs_release<C::REGS_CTRL>();
 
   if (warp == 0) {
     // ======================= TMA producer
@@ -164,9 +186,8 @@ __global__ void __launch_bounds__(384, 1)
         filled = j + 1;
       }
       // Drain: wait (bounded) for the copies this thread issued, so none lands after exit.
-      WaitCtl drain{abort_flag, p.status, p.timeout_ns};
       volatile int zero = 0;
-      drain.abort_flag = &zero;
+      WaitCtl drain{&zero, p.status, p.timeout_ns};
       mbar_wait(bar(C::BAR_Q), 0, drain);
       for (int j = max(0, filled - C::STAGES); j < filled; ++j) {
         const int s = j % C::STAGES;
@@ -181,6 +202,7 @@ __global__ void __launch_bounds__(384, 1)
       constexpr uint32_t IDESC_O = idesc_bf16_f32(C::BM, D, 0, 1);
       const uint32_t col_s[2] = {C::COL_S0, C::COL_S1};
       const uint32_t col_o[2] = {C::COL_O0, C::COL_O1};
+      const uint32_t col_p[2] = {C::COL_P0, C::COL_P1};
       bool ok = mbar_wait(bar(C::BAR_Q), 0, ctl);
       auto issue_s = [&](int k, int s) {
         const uint32_t qa = sbase + C::OFF_Q + k * C::Q_BYTES;
@@ -197,7 +219,7 @@ __global__ void __launch_bounds__(384, 1)
         const uint32_t va = sbase + C::OFF_V + s * C::KV_BYTES;
 #pragma unroll
         for (int kk = 0; kk < C::BN / 16; ++kk) {
-          umma_ts(tmem + col_o[k], tmem + col_s[k] + kk * 8, sdesc_sw128(va + kk * 16 * 128, C::CHUNK_KV, 1024),
+          umma_ts(tmem + col_o[k], tmem + col_p[k] + kk * 8, sdesc_sw128(va + kk * 16 * 128, C::CHUNK_KV, 1024),
                   IDESC_O, (j > 0 || kk > 0) ? 1u : 0u);
         }
       };
@@ -217,41 +239,68 @@ __global__ void __launch_bounds__(384, 1)
         const uint32_t ph = (j / C::STAGES) & 1;
         const int s1 = (j + 1) % C::STAGES;
         const uint32_t ph1 = ((j + 1) / C::STAGES) & 1;
-        if (!mbar_wait(bar(C::BAR_VF + s), ph, ctl)) { ok = false; break; }
-        for (int k = 0; k < 2 && ok; ++k) {
-          if (j >= n_kv[k]) continue;
-          if (!mbar_wait(bar(C::BAR_P + k), j & 1, ctl)) { ok = false; break; }
-          tc_fence_after();
-          issue_pv(k, s, j);
-          if (j == n_kv[k] - 1) {
-            umma_commit(bar(C::BAR_O + k));
-          } else {
-            if (!mbar_wait(bar(C::BAR_KF + s1), ph1, ctl)) { ok = false; break; }
+        if constexpr (C::SEP_P) {
+          // S_k(j+1) as soon as softmax k has read S_k(j): overlaps softmax k(j).
+          for (int k = 0; k < 2 && ok; ++k) {
+            if (j + 1 >= n_kv[k]) continue;
+            if (!mbar_wait(bar(C::BAR_SFREE + k), j & 1, ctl) || !mbar_wait(bar(C::BAR_KF + s1), ph1, ctl)) {
+              ok = false;
+              break;
+            }
             tc_fence_after();
             issue_s(k, s1);
             umma_commit(bar(C::BAR_S + k));
+          }
+          if (!ok || !mbar_wait(bar(C::BAR_VF + s), ph, ctl)) { ok = false; break; }
+          for (int k = 0; k < 2 && ok; ++k) {
+            if (j >= n_kv[k]) continue;
+            if (!mbar_wait(bar(C::BAR_P + k), j & 1, ctl)) { ok = false; break; }
+            tc_fence_after();
+            issue_pv(k, s, j);
+            umma_commit(bar(C::BAR_PV + k));
+            if (j == n_kv[k] - 1) umma_commit(bar(C::BAR_O + k));
+          }
+        } else {
+          // P lives over S_k: S_k(j+1) may only follow PV_k(j) (MMAs run in issue order).
+          if (!mbar_wait(bar(C::BAR_VF + s), ph, ctl)) { ok = false; break; }
+          for (int k = 0; k < 2 && ok; ++k) {
+            if (j >= n_kv[k]) continue;
+            if (!mbar_wait(bar(C::BAR_P + k), j & 1, ctl)) { ok = false; break; }
+            tc_fence_after();
+            issue_pv(k, s, j);
+            umma_commit(bar(C::BAR_PV + k));
+            if (j == n_kv[k] - 1) {
+              umma_commit(bar(C::BAR_O + k));
+            } else {
+              if (!mbar_wait(bar(C::BAR_KF + s1), ph1, ctl)) { ok = false; break; }
+              tc_fence_after();
+              issue_s(k, s1);
+              umma_commit(bar(C::BAR_S + k));
+            }
           }
         }
         umma_commit(bar(C::BAR_KVE + s));
       }
       // Drain: every MMA issued above has finished before TMEM is released.
       umma_commit(bar(C::BAR_DRAIN));
-      WaitCtl drain{abort_flag, p.status, p.timeout_ns};
       volatile int zero = 0;
-      drain.abort_flag = &zero;
+      WaitCtl drain{&zero, p.status, p.timeout_ns};
       mbar_wait(bar(C::BAR_DRAIN), 0, drain);
     }
   } else if (warp >= 4) {
     // ======================= softmax + epilogue, one thread per tile row
+    regs_claim<C::REGS_SOFTMAX>();
     const int k = (warp - 4) >> 2;
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
     const uint32_t lane_base = tmem + (uint32_t(quarter * 32) << 16);
     const uint32_t s_addr = lane_base + (k ? C::COL_S1 : C::COL_S0);
     const uint32_t o_addr = lane_base + (k ? C::COL_O1 : C::COL_O0);
+    const uint32_t p_addr = lane_base + (k ? C::COL_P1 : C::COL_P0);
     const int token = t0[k] + (row >> p.log2P);
     const int head = head0 + (row & (p.P - 1));
     const float sl2 = p.scale_log2;
+    const float2 sl2x2 = make_float2(sl2, sl2);
     const int nk = n_kv[k];
     const int t_first = t0[k];
     float m = -INFINITY, l = 0.f;
@@ -261,14 +310,16 @@ __global__ void __launch_bounds__(384, 1)
       tc_fence_after();
       float s[128];
       {
-        uint32_t r[64];
-        tmem_ld64(s_addr, r);
+        uint32_t r[128];
+        tmem_ld128(s_addr, r);
 #pragma unroll
-        for (int u = 0; u < 64; ++u) s[u] = __uint_as_float(r[u]);
-        tmem_ld64(s_addr + 64, r);
-#pragma unroll
-        for (int u = 0; u < 64; ++u) s[64 + u] = __uint_as_float(r[u]);
+        for (int u = 0; u < 128; ++u) s[u] = __uint_as_float(r[u]);
       }
+      // S_k is in registers: the next S_k may be written.
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(C::BAR_SFREE + k));
+
       const int key0 = j * C::BN;
       const bool tail = key0 + C::BN > p.N;
       const bool diag = p.causal && (key0 + C::BN - 1 > t_first);
@@ -278,9 +329,17 @@ __global__ void __launch_bounds__(384, 1)
         for (int u = 0; u < 128; ++u)
           if (key0 + u > lim) s[u] = -INFINITY;
       }
-      float mx = s[0];
+      // row maximum: eight independent 3-input chains, then a short tree
+      float m8[8];
 #pragma unroll
-      for (int u = 1; u < 128; ++u) mx = fmaxf(mx, s[u]);
+      for (int i = 0; i < 8; ++i) m8[i] = fmax3(s[i], s[8 + i], s[16 + i]);
+#pragma unroll
+      for (int u = 24; u < 120; u += 16)
+#pragma unroll
+        for (int i = 0; i < 8; ++i) m8[i] = fmax3(m8[i], s[u + i], s[u + 8 + i]);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) m8[i] = fmaxf(m8[i], s[120 + i]);
+      const float mx = fmax3(fmax3(m8[0], m8[1], m8[2]), fmax3(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7]));
       const float m_new = fmaxf(m, mx);
       // Keep the stale maximum unless it grew by more than 2^8 in the exp2
       // domain: O / l is exact either way, and P stays <= 256.
@@ -288,23 +347,38 @@ __global__ void __launch_bounds__(384, 1)
       const float m_use = need ? m_new : m;
       const float f = (need && j > 0) ? ex2_approx((m - m_new) * sl2) : 1.0f;
       const bool rescale = (j > 0) && __any_sync(0xffffffffu, need);
-      const float ms = m_use * sl2;
-      float lsum = 0.f;
+      const float2 nms = make_float2(-m_use * sl2, -m_use * sl2);
+      float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
-      for (int u = 0; u < 128; ++u) {
-        s[u] = ex2_approx(fmaf(s[u], sl2, -ms));
-        lsum += s[u];
+      for (int u = 0; u < 64; ++u) {
+        const float2 x = ffma2(make_float2(s[2 * u], s[2 * u + 1]), sl2x2, nms);
+        float2 e;
+        if ((u & 7) < EMU) {
+          e = exp2_poly2(x);
+        } else {
+          e.x = ex2_approx(x.x);
+          e.y = ex2_approx(x.y);
+        }
+        acc[u & 3] = fadd2(acc[u & 3], e);
+        s[2 * u] = e.x;
+        s[2 * u + 1] = e.y;
       }
-      l = l * f + lsum;
+      const float2 a01 = fadd2(acc[0], acc[1]), a23 = fadd2(acc[2], acc[3]);
+      const float2 a = fadd2(a01, a23);
+      l = l * f + (a.x + a.y);
+      // P_k and O_k are free once PV_k(j-1) has completed.
+      if (j > 0) {
+        if (!mbar_wait_warp(bar(C::BAR_PV + k), (j - 1) & 1, ctl)) { ok = false; break; }
+        tc_fence_after();
+      }
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
         uint32_t r[32];
 #pragma unroll
         for (int u = 0; u < 32; ++u) r[u] = pack_bf16x2(s[c * 64 + 2 * u], s[c * 64 + 2 * u + 1]);
-        tmem_st32(s_addr + c * 32, r);
+        tmem_st32(p_addr + c * 32, r);
       }
       if (rescale) {
-        // O holds PV up to tile j-1 (complete: S_j was committed after it).
 #pragma unroll 1
         for (int c = 0; c < D; c += 32) {
           uint32_t r[32];

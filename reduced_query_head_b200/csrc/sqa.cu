@@ -7,6 +7,7 @@
 #include <climits>
 #include <cmath>
 #include <cstdint>
+#include <cstdlib>
 #include <mutex>
 
 #include "sqa.h"
@@ -36,6 +37,37 @@ struct DeviceState {
   int sms = 0;
 };
 
+// Attention kernels by the share of exp2 evaluated on the FMA pipe (eighths
+// of the column pairs; the rest use the MUFU unit).
+using AttnKernel = void (*)(const CUtensorMap, const CUtensorMap, const CUtensorMap, const AttnParams);
+constexpr int kEmuChoices[] = {0, 2, 3, 4, 5};
+constexpr int kNumEmu = 5;
+AttnKernel attn_kernel_64(int i) {
+  static const AttnKernel t[kNumEmu] = {sqa::attn_fwd_kernel<64, 0>, sqa::attn_fwd_kernel<64, 2>,
+                                        sqa::attn_fwd_kernel<64, 3>, sqa::attn_fwd_kernel<64, 4>,
+                                        sqa::attn_fwd_kernel<64, 5>};
+  return t[i];
+}
+AttnKernel attn_kernel_128(int i) {
+  static const AttnKernel t[kNumEmu] = {sqa::attn_fwd_kernel<128, 0>, sqa::attn_fwd_kernel<128, 2>,
+                                        sqa::attn_fwd_kernel<128, 3>, sqa::attn_fwd_kernel<128, 4>,
+                                        sqa::attn_fwd_kernel<128, 5>};
+  return t[i];
+}
+// Default split per head size; SQA_EXP2_POLY_EIGHTHS=<0|2|3|4|5> overrides it.
+constexpr int kDefaultEmu64 = 3, kDefaultEmu128 = 2;
+int emu_index(int d) {
+  int want = d == 64 ? kDefaultEmu64 : kDefaultEmu128;
+  if (const char* e = getenv("SQA_EXP2_POLY_EIGHTHS")) {
+    const int v = atoi(e);
+    for (int i = 0; i < kNumEmu; ++i)
+      if (kEmuChoices[i] == v) want = v;
+  }
+  for (int i = 0; i < kNumEmu; ++i)
+    if (kEmuChoices[i] == want) return i;
+  return 0;
+}
+
 std::mutex g_mu;
 DeviceState g_dev[kMaxDevices];
 EncodeTiledFn g_encode = nullptr;
@@ -59,11 +91,22 @@ int device_state(DeviceState** out) {
     }
     if (cudaGetSymbolAddress(reinterpret_cast<void**>(&st.status), g_sqa_status) != cudaSuccess) return SQA_ERR_CUDA;
     if (cudaDeviceGetAttribute(&st.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return SQA_ERR_CUDA;
-    if (cudaFuncSetAttribute(sqa::attn_fwd_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             AttnCfg<64>::SMEM_BYTES) != cudaSuccess ||
-        cudaFuncSetAttribute(sqa::attn_fwd_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             AttnCfg<128>::SMEM_BYTES) != cudaSuccess ||
-        cudaFuncSetAttribute(sqa::gemm_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    for (int e = 0; e < kNumEmu; ++e) {
+      if (cudaFuncSetAttribute(attn_kernel_64(e), cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               AttnCfg<64>::SMEM_BYTES) != cudaSuccess ||
+          cudaFuncSetAttribute(attn_kernel_128(e), cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               AttnCfg<128>::SMEM_BYTES) != cudaSuccess)
+        return SQA_ERR_CUDA;
+      // The kernels re-split their registers between warpgroups at run time;
+      // the split is only valid for the per-thread count they were built for.
+      cudaFuncAttributes a64, a128;
+      if (cudaFuncGetAttributes(&a64, attn_kernel_64(e)) != cudaSuccess ||
+          cudaFuncGetAttributes(&a128, attn_kernel_128(e)) != cudaSuccess)
+        return SQA_ERR_CUDA;
+      if (a64.numRegs != AttnCfg<64>::REGS_LAUNCH || a128.numRegs != AttnCfg<128>::REGS_LAUNCH)
+        return SQA_ERR_UNSUPPORTED;
+    }
+    if (cudaFuncSetAttribute(sqa::gemm_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              GemmCfg::SMEM_BYTES) != cudaSuccess)
       return SQA_ERR_CUDA;
     st.ready = true;
@@ -150,7 +193,8 @@ int launch_attn(const DeviceState* st, const void* q, const void* k, const void*
   p.scale_log2 = (float)((double)scale * 1.4426950408889634);  // scale * log2(e)
   p.status = st->status;
   p.timeout_ns = g_wait_ns.load();
-  sqa::attn_fwd_kernel<D><<<(unsigned)grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);
+  const AttnKernel kern = D == 64 ? attn_kernel_64(emu_index(D)) : attn_kernel_128(emu_index(D));
+  kern<<<(unsigned)grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);
   return cudaGetLastError() == cudaSuccess ? SQA_OK : SQA_ERR_CUDA;
 }
 
