@@ -48,11 +48,11 @@ def assert_close(got, want, what="", out_rounding=False):
     return max_abs, rel
 
 
-def attn_inputs(B, N, H_q, H_kv, d, seed=0, factor=1.0):
+def attn_inputs(B, N, H_q, H_kv, d, seed=0, factor=1.0, v_factor=None):
     """bf16 bit arrays q [B,N,H_q,d], k/v [B,N,H_kv,d] from the seeded generator."""
     q = synth.bf16_bits((B, N, H_q, d), seed, "q", factor)
     k = synth.bf16_bits((B, N, H_kv, d), seed, "k", factor)
-    v = synth.bf16_bits((B, N, H_kv, d), seed, "v", factor)
+    v = synth.bf16_bits((B, N, H_kv, d), seed, "v", factor if v_factor is None else v_factor)
     return q, k, v
 
 

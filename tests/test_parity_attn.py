@@ -16,9 +16,10 @@ from helpers import (HEAD_CONFIGS_32K, LONG_HEAD_CONFIGS, assert_close, attn_inp
 pytestmark = pytest.mark.gpu
 
 
-def _full_check(B, N, H_q, H_kv, d, causal, scale=None, seed=0, factor=1.0, what="", out_rounding=True):
+def _full_check(B, N, H_q, H_kv, d, causal, scale=None, seed=0, factor=1.0, what="", out_rounding=True,
+                v_factor=None):
     scale = default_scale(d) if scale is None else scale
-    qb, kb, vb = attn_inputs(B, N, H_q, H_kv, d, seed, factor)
+    qb, kb, vb = attn_inputs(B, N, H_q, H_kv, d, seed, factor, v_factor)
     out = bf16_tensor_to_f64(run_attn(qb, kb, vb, causal, scale))
     want = oracle.attention(oracle.widen_bf16(qb), oracle.widen_bf16(kb), oracle.widen_bf16(vb), causal, scale)
     return assert_close(out, want, what or str((B, N, H_q, H_kv, d, causal)), out_rounding=out_rounding)
@@ -75,10 +76,11 @@ def test_nondefault_scale(scale):
     _full_check(1, 300, 4, 2, 128, False, scale=scale, seed=4)
 
 
-def test_large_scores_stress_rescale():
-    # values x4 make score rows peaky, so the running max moves by > 2^8 often
-    _full_check(1, 2048, 4, 1, 64, False, seed=5, factor=2.0)
-    _full_check(1, 2048, 4, 1, 128, True, seed=6, factor=2.0)
+def test_peaky_scores_exercise_rescale():
+    # q, k x2 give score rows with std ~4 (x1.44 in the exp2 domain), so the
+    # running maximum often moves by more than 2^8 and O is rescaled
+    _full_check(1, 2048, 4, 1, 64, False, seed=5, factor=2.0, v_factor=1.0)
+    _full_check(1, 2048, 4, 1, 128, True, seed=6, factor=2.0, v_factor=1.0)
 
 
 def test_deterministic_bitwise():
