@@ -365,6 +365,17 @@ def bench_extra(args):
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
     peaks = load_peaks()
     lines = []
+    clocks = ClockSampler(0)
+    clocks.start()
+    try:
+        _bench_extra(args, sqa, torch, device, stream, flush, peaks, lines)
+    finally:
+        clk = clocks.stop()
+    print(json.dumps({"workload": args.workload, "clocks": clk}), flush=True)
+    return lines
+
+
+def _bench_extra(args, sqa, torch, device, stream, flush, peaks, lines):
     if args.workload in ("long", "sweep"):
         if args.workload == "long":
             grid = [(N, H_q, H_kv, 64, c, 1.0, 0) for N in (65536, 131072, 200000)
@@ -440,7 +451,6 @@ def bench_extra(args):
         fl_gemm = 2.0 * M * dm * (H_q + 2 * H_kv) * d + 2.0 * M * (H_q * d) * dm
         med = statistics.median(ms)
         # per-kernel split
-        Q = ws[:0]
         qkv = torch.empty((M, (H_q + 2 * H_kv) * d), dtype=torch.bfloat16, device=device)
         wqkv = torch.cat([wq, wk, wv], 0).contiguous()
         ms_qkv = statistics.median(_time_launches(

@@ -29,6 +29,9 @@ serve as the dot-product step; nothing else is blocked, fused or reordered.
 """
 from __future__ import annotations
 
+import os
+from concurrent.futures import ThreadPoolExecutor
+
 import numpy as np
 
 __all__ = [
@@ -138,14 +141,38 @@ def attention_rows(q_rows, k, v, rows, N: int, causal: bool, scale: float, chunk
     H_q = q_rows.shape[1]
     out = np.empty((len(rows), H_q, d), dtype=np.float64)
     bs, ts = rows // N, rows % N
-    for b in np.unique(bs):
+
+    def one_head(b, i):
         sel = np.nonzero(bs == b)[0]
-        for i in range(H_q):
-            g = group_of_head(i, H_q, H_kv)
-            kh = np.asarray(k[b, :, g, :], dtype=np.float64).copy()
-            vh = np.asarray(v[b, :, g, :], dtype=np.float64).copy()
-            out[sel, i, :] = _head_rows(q_rows[sel, i, :], kh, vh, ts[sel], causal, scale, chunk)
+        g = group_of_head(i, H_q, H_kv)
+        kh = np.asarray(k[b, :, g, :], dtype=np.float64).copy()   # explicit repetition
+        vh = np.asarray(v[b, :, g, :], dtype=np.float64).copy()
+        out[sel, i, :] = _head_rows(q_rows[sel, i, :], kh, vh, ts[sel], causal, scale, chunk)
+
+    # (batch, head) pairs are independent: run them on a thread pool
+    _map_pairs(one_head, [(int(b), i) for b in np.unique(bs) for i in range(H_q)])
     return out
+
+
+def _map_pairs(fn, pairs):
+    """Apply fn(*pair) to independent work items; threads when there are several."""
+    workers = min(len(pairs), os.cpu_count() or 1)
+    if workers <= 1:
+        for pr in pairs:
+            fn(*pr)
+        return
+    try:
+        from threadpoolctl import threadpool_limits
+        limit = threadpool_limits(limits=1, user_api="blas")
+    except Exception:   # pragma: no cover - threadpoolctl is optional
+        limit = None
+    try:
+        with ThreadPoolExecutor(max_workers=workers) as ex:
+            for f in [ex.submit(fn, *pr) for pr in pairs]:
+                f.result()
+    finally:
+        if limit is not None:
+            limit.restore_original_limits()
 
 
 def linear(x: np.ndarray, w: np.ndarray) -> np.ndarray:
