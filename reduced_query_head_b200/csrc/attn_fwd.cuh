@@ -12,18 +12,15 @@
 // dividing H_q/H_kv), stacked so that tile row r = token_local * P + head
 // offset: every key/value tile brought into shared memory serves all P heads.
 //
-// Warp roles (20 warps):
+// Warp roles (12 warps):
 //   warp 0   TMA producer: Q0/Q1 once, then K_j and V_j into a ring of stages
 //   warp 1   MMA issuer: S_k = Q_k K_j^T into TMEM, O_k += P_k V_j from TMEM
 //   warp 2   owns the TMEM allocation
-//   warps 4-11 / 12-19  softmax for tile 0 / tile 1. Each tile row (TMEM lane)
-//            has two threads, one per 64-key half of a step; they exchange
-//            their half-row maxima through shared memory. Online softmax with
-//            a lazily rescaled running max, P written back to TMEM as bf16,
-//            epilogue O / l -> bf16 -> global.
+//   warps 4-7 / 8-11  softmax for tile 0 / tile 1 (thread = row = TMEM lane):
+//            online softmax with a lazily rescaled running max, P written
+//            back to TMEM as bf16 over S, epilogue O / l -> bf16 -> global.
 //
-// TMEM columns: S0 [0,128), S1 [128,256), O0 [256,256+D), O1 [256+D,256+2D);
-// P0/P1 after O1 at d=64, over the first half of S0/S1 at d=128.
+// TMEM columns: S0 [0,128), S1 [128,256), O0 [256,256+D), O1 [256+D,256+2D).
 // Every wait is bounded; on time-out the kernel records the status, drains
 // its own copies and MMAs, frees TMEM and returns.
 #pragma once
@@ -74,16 +71,11 @@ struct AttnCfg {
   static constexpr int BAR_PV = BAR_P + 2;              // [2] O_k += P_k V done
   static constexpr int BAR_O = BAR_PV + 2;              // [2] last PV of tile k done
   static constexpr int BAR_DRAIN = BAR_O + 2;
-  static constexpr int BAR_X = BAR_DRAIN + 1;           // [2 tiles][4 quarters] half-row exchange (2 warps)
-  static constexpr int N_BARS = BAR_X + 8;
+  static constexpr int N_BARS = BAR_DRAIN + 1;
   static constexpr int OFF_MISC = OFF_BAR + N_BARS * 8;  // tmem base (u32), abort flag (u32)
-  // row-max exchange between the two half-row threads: [step parity][tile][half][row]
-  static constexpr int OFF_XMAX = (OFF_MISC + 16 + 15) & ~15;
-  static constexpr int OFF_XL = OFF_XMAX + 2 * 2 * 2 * 128 * 4;  // final row sums [tile][half][row]
-  static constexpr int SMEM_BYTES = OFF_XL + 2 * 2 * 128 * 4 + 1024;  // + alignment slack
-  // warpgroup 0: control; warpgroups 1..4: softmax (tile k = wg-1 >> 1, column half = wg-1 & 1)
-  static constexpr int THREADS = 640;
-  static constexpr int REGS_LAUNCH = 96, REGS_CTRL = 56, REGS_SOFTMAX = 104;
+  static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;  // + alignment slack
+  static constexpr int THREADS = 384;
+  static constexpr int REGS_LAUNCH = 168, REGS_CTRL = 56, REGS_SOFTMAX = 224;
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr uint32_t COL_S0 = 0, COL_S1 = 128;
   static constexpr uint32_t COL_O0 = 256, COL_O1 = 256 + D;
@@ -95,7 +87,7 @@ struct AttnCfg {
 // EMU: of every 8 column pairs of a score row, how many take 2^x from the
 // polynomial on the FMA pipe instead of the MUFU unit (0..8).
 template <int D, int EMU>
-__global__ void __launch_bounds__(640, 1)
+__global__ void __launch_bounds__(384, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
   using C = AttnCfg<D>;
@@ -142,8 +134,7 @@ __global__ void __launch_bounds__(640, 1)
   if (tid == 0) {
     for (int i = 0; i < C::N_BARS; ++i) {
       const bool per_warp = (i >= C::BAR_SFREE && i < C::BAR_SFREE + 2) || (i >= C::BAR_P && i < C::BAR_P + 2);
-      const bool pair = i >= C::BAR_X;
-      mbar_init(bar(i), per_warp ? 8 : pair ? 2 : 1);   // 8 softmax warps per tile; 2 warps per row pair
+      mbar_init(bar(i), per_warp ? 4 : 1);
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -159,9 +150,9 @@ __global__ void __launch_bounds__(640, 1)
 
   // Register split: the kernel launches with REGS_LAUNCH per thread (the host
   // checks this before launching). Warpgroup 0 (producer, MMA, TMEM owner)
-  // gives registers back, the four softmax warpgroups take some of them:
-  // 128*REGS_CTRL + 512*REGS_SOFTMAX <= 640*REGS_LAUNCH.
-  static_assert(128 * C::REGS_CTRL + 512 * C::REGS_SOFTMAX <= 640 * C::REGS_LAUNCH, "register split");
+  // gives registers back, the two softmax warpgroups take them:
+  // 128*REGS_CTRL + 256*REGS_SOFTMAX == 384*REGS_LAUNCH.
+  static_assert(128 * C::REGS_CTRL + 256 * C::REGS_SOFTMAX == 384 * C::REGS_LAUNCH, "register split");
   if (warp < 4) regs_release<C::REGS_CTRL>();
 
   if (warp == 0) {
@@ -297,21 +288,15 @@ __global__ void __launch_bounds__(640, 1)
       mbar_wait(bar(C::BAR_DRAIN), 0, drain);
     }
   } else if (warp >= 4) {
-    // ======================= softmax + epilogue
-    // Two threads per tile row: column half h of the 128 keys of each step.
+    // ======================= softmax + epilogue, one thread per tile row
     regs_claim<C::REGS_SOFTMAX>();
-    const int sw = warp - 4;
-    const int k = sw >> 3;                 // query tile
-    const int h = (sw >> 2) & 1;           // key-column half
-    const int quarter = warp & 3;          // TMEM lane quarter
+    const int k = (warp - 4) >> 2;
+    const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
-    const uint32_t xbar = bar(C::BAR_X + k * 4 + quarter);  // this row's two warps
     const uint32_t lane_base = tmem + (uint32_t(quarter * 32) << 16);
-    const uint32_t s_addr = lane_base + (k ? C::COL_S1 : C::COL_S0) + h * 64;
-    const uint32_t o_addr = lane_base + (k ? C::COL_O1 : C::COL_O0) + h * (D / 2);
-    const uint32_t p_addr = lane_base + (k ? C::COL_P1 : C::COL_P0) + h * 32;
-    float* xmax = reinterpret_cast<float*>(smem + C::OFF_XMAX);
-    float* xl = reinterpret_cast<float*>(smem + C::OFF_XL);
+    const uint32_t s_addr = lane_base + (k ? C::COL_S1 : C::COL_S0);
+    const uint32_t o_addr = lane_base + (k ? C::COL_O1 : C::COL_O0);
+    const uint32_t p_addr = lane_base + (k ? C::COL_P1 : C::COL_P0);
     const int token = t0[k] + (row >> p.log2P);
     const int head = head0 + (row & (p.P - 1));
     const float sl2 = p.scale_log2;
@@ -323,64 +308,49 @@ __global__ void __launch_bounds__(640, 1)
     for (int j = 0; j < nk; ++j) {
       if (!mbar_wait_warp(bar(C::BAR_S + k), j & 1, ctl)) { ok = false; break; }
       tc_fence_after();
-      float s[64];
+      float s[128];
       {
-        uint32_t r[64];
-        tmem_ld64x(s_addr, r);
+        uint32_t r[128];
+        tmem_ld128(s_addr, r);
 #pragma unroll
-        for (int u = 0; u < 64; ++u) s[u] = __uint_as_float(r[u]);
+        for (int u = 0; u < 128; ++u) s[u] = __uint_as_float(r[u]);
       }
-      // this half of S_k is in registers
+      // S_k is in registers: the next S_k may be written.
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(C::BAR_SFREE + k));
 
-      const int key0 = j * C::BN + h * 64;
-      const bool tail = key0 + 64 > p.N;
-      const bool diag = p.causal && (key0 + 63 > t_first);
+      const int key0 = j * C::BN;
+      const bool tail = key0 + C::BN > p.N;
+      const bool diag = p.causal && (key0 + C::BN - 1 > t_first);
       if (tail || diag) {
         const int lim = p.causal ? min(token, p.N - 1) : p.N - 1;  // last visible key
 #pragma unroll
-        for (int u = 0; u < 64; ++u)
+        for (int u = 0; u < 128; ++u)
           if (key0 + u > lim) s[u] = -INFINITY;
       }
-      // half-row maximum: eight independent 3-input chains, then a short tree
+      // row maximum: eight independent 3-input chains, then a short tree
       float m8[8];
 #pragma unroll
       for (int i = 0; i < 8; ++i) m8[i] = fmax3(s[i], s[8 + i], s[16 + i]);
 #pragma unroll
-      for (int u = 24; u < 56; u += 16)
+      for (int u = 24; u < 120; u += 16)
 #pragma unroll
         for (int i = 0; i < 8; ++i) m8[i] = fmax3(m8[i], s[u + i], s[u + 8 + i]);
 #pragma unroll
-      for (int i = 0; i < 8; ++i) m8[i] = fmaxf(m8[i], s[56 + i]);
-      const float mh = fmax3(fmax3(m8[0], m8[1], m8[2]), fmax3(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7]));
-      // Exchange with the other half of the row through shared memory, the
-      // two warps meeting on an mbarrier (bounded wait; phase j). The buffer
-      // is double-buffered by step parity: the partner has read step j's value
-      // before it arrives for step j+1, which this warp waits for before it
-      // writes step j+2.
-      float* xm = xmax + ((j & 1) * 4 + k * 2) * 128;
-      xm[h * 128 + row] = mh;
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(xbar);
-      if (!mbar_wait_warp(xbar, j & 1, ctl)) { ok = false; break; }
-      tc_fence_after();
-      const float mx = fmaxf(mh, xm[(h ^ 1) * 128 + row]);
+      for (int i = 0; i < 8; ++i) m8[i] = fmaxf(m8[i], s[120 + i]);
+      const float mx = fmax3(fmax3(m8[0], m8[1], m8[2]), fmax3(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7]));
       const float m_new = fmaxf(m, mx);
       // Keep the stale maximum unless it grew by more than 2^8 in the exp2
-      // domain: O / l is exact either way, and P stays <= 256. Both halves of
-      // a row see the same maxima, so they take the same decisions.
+      // domain: O / l is exact either way, and P stays <= 256.
       const bool need = (j == 0) || ((m_new - m) * sl2 > 8.0f);
       const float m_use = need ? m_new : m;
       const float f = (need && j > 0) ? ex2_approx((m - m_new) * sl2) : 1.0f;
       const bool rescale = (j > 0) && __any_sync(0xffffffffu, need);
       const float2 nms = make_float2(-m_use * sl2, -m_use * sl2);
       float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-      uint32_t pk[32];
 #pragma unroll
-      for (int u = 0; u < 32; ++u) {
+      for (int u = 0; u < 64; ++u) {
         const float2 x = ffma2(make_float2(s[2 * u], s[2 * u + 1]), sl2x2, nms);
         float2 e;
         if ((u & 7) < EMU) {
@@ -390,7 +360,8 @@ __global__ void __launch_bounds__(640, 1)
           e.y = ex2_approx(x.y);
         }
         acc[u & 3] = fadd2(acc[u & 3], e);
-        pk[u] = pack_bf16x2(e.x, e.y);
+        s[2 * u] = e.x;
+        s[2 * u + 1] = e.y;
       }
       const float2 a01 = fadd2(acc[0], acc[1]), a23 = fadd2(acc[2], acc[3]);
       const float2 a = fadd2(a01, a23);
@@ -400,15 +371,21 @@ __global__ void __launch_bounds__(640, 1)
         if (!mbar_wait_warp(bar(C::BAR_PV + k), (j - 1) & 1, ctl)) { ok = false; break; }
         tc_fence_after();
       }
-      tmem_st32(p_addr, pk);
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        uint32_t r[32];
+#pragma unroll
+        for (int u = 0; u < 32; ++u) r[u] = pack_bf16x2(s[c * 64 + 2 * u], s[c * 64 + 2 * u + 1]);
+        tmem_st32(p_addr + c * 32, r);
+      }
       if (rescale) {
 #pragma unroll 1
-        for (int c = 0; c < D / 2; c += 16) {
-          uint32_t r[16];
-          tmem_ld16(o_addr + c, r);
+        for (int c = 0; c < D; c += 32) {
+          uint32_t r[32];
+          tmem_ld32(o_addr + c, r);
 #pragma unroll
-          for (int u = 0; u < 16; ++u) r[u] = __float_as_uint(__uint_as_float(r[u]) * f);
-          tmem_st16(o_addr + c, r);
+          for (int u = 0; u < 32; ++u) r[u] = __float_as_uint(__uint_as_float(r[u]) * f);
+          tmem_st32(o_addr + c, r);
         }
       }
       tmem_st_wait();
@@ -417,35 +394,24 @@ __global__ void __launch_bounds__(640, 1)
       if (lane == 0) mbar_arrive(bar(C::BAR_P + k));
       m = m_use;
     }
-    // Row sum = the two halves' sums (same maximum trajectory): one more
-    // exchange, phase nk of the pair barrier.
-    float l_row = l;
-    if (ok && nk > 0) {
-      xl[(k * 2 + h) * 128 + row] = l;
-      __syncwarp();
-      if (lane == 0) mbar_arrive(xbar);
-      ok = mbar_wait_warp(xbar, nk & 1, ctl);
-      l_row = l + xl[(k * 2 + (h ^ 1)) * 128 + row];
-    }
     if (ok && nk > 0 && mbar_wait_warp(bar(C::BAR_O + k), 0, ctl)) {
       tc_fence_after();
-      const float inv_l = 1.0f / l_row;
+      const float inv_l = 1.0f / l;
       const bool store = token < p.N;
-      __nv_bfloat16* dst =
-          p.out + (((size_t)b * p.N + (store ? token : 0)) * p.H_q + head) * D + h * (D / 2);
+      __nv_bfloat16* dst = p.out + (((size_t)b * p.N + (store ? token : 0)) * p.H_q + head) * D;
 #pragma unroll
-      for (int c = 0; c < D / 2; c += 16) {
-        uint32_t r[16];
-        tmem_ld16(o_addr + c, r);  // all lanes: the load is warp-collective
-        uint4 w[2];
+      for (int c = 0; c < D; c += 32) {
+        uint32_t r[32];
+        tmem_ld32(o_addr + c, r);  // all lanes: the load is warp-collective
+        uint4 w[4];
         uint32_t* wp = reinterpret_cast<uint32_t*>(w);
 #pragma unroll
-        for (int u = 0; u < 8; ++u)
+        for (int u = 0; u < 16; ++u)
           wp[u] = pack_bf16x2(__uint_as_float(r[2 * u]) * inv_l, __uint_as_float(r[2 * u + 1]) * inv_l);
         if (store) {
           uint4* d4 = reinterpret_cast<uint4*>(dst + c);
-          d4[0] = w[0];
-          d4[1] = w[1];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) d4[u] = w[u];
         }
       }
     }
