@@ -150,12 +150,15 @@ def bench_sqa(args):
     stream = torch.cuda.current_stream()
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
 
-    # Each rank runs its own independent copy of the workload (weak scaling; the
-    # seed differs per rank so ranks do not compute identical problems).
+    # The global workload is `world` independent sequences (one batch element
+    # per GPU); attention over (batch, group) units needs no exchange, so each
+    # rank runs its own shard (weak scaling). The seed is the global batch index.
+    from reduced_query_head_b200.dist import max_over_ranks, shard_range
+    b_lo, b_hi = shard_range(world, rank, world)
     cfgs = []
     for name, H_q, H_kv in HEAD_CONFIGS_32K:
-        B, N, d = 1, 32768, 64
-        host, dev = make_attn_inputs(B, N, H_q, H_kv, d, rank, 1.0, device, pinned_host=True)
+        B, N, d = b_hi - b_lo, 32768, 64
+        host, dev = make_attn_inputs(B, N, H_q, H_kv, d, b_lo, 1.0, device, pinned_host=True)
         out = torch.empty((B, N, H_q, d), dtype=torch.bfloat16, device=device)
         out_host = torch.empty((B, N, H_q, d), dtype=torch.bfloat16, pin_memory=True)
         cfgs.append(dict(name=name, B=B, N=N, H_q=H_q, H_kv=H_kv, d=d, host=host, dev=dev, out=out,
@@ -219,10 +222,7 @@ def bench_sqa(args):
     torch.cuda.synchronize()
     e2e_ms = sum(a.elapsed_time(b) for a, b in e2e_ev) / args.steps
 
-    t_local = torch.tensor([step_ms, e2e_ms], dtype=torch.float64, device=device)
-    if world > 1:
-        dist.all_reduce(t_local, op=dist.ReduceOp.MAX)
-    step_ms_max, e2e_ms_max = float(t_local[0]), float(t_local[1])
+    step_ms_max, e2e_ms_max = max_over_ranks([step_ms, e2e_ms], device=device)
 
     value = flops_step * world / (step_ms_max * 1e-3) / 1e12
     e2e_value = flops_step * world / (e2e_ms_max * 1e-3) / 1e12

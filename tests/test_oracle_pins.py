@@ -55,6 +55,13 @@ def test_group_map_matches_gqa_diagram():
         assert got == case["groups"]
 
 
+def test_repeat_kv_matches_numpy_repeat():
+    kv = _rand((2, 3, 4, 5), 45)
+    assert np.array_equal(oracle.repeat_kv(kv, 8), np.repeat(kv, 2, axis=2))
+    assert np.array_equal(oracle.repeat_kv(kv, 4), kv)
+    assert np.array_equal(oracle.repeat_kv(kv[:, :, :1], 3), np.repeat(kv[:, :, :1], 3, axis=2))
+
+
 def test_group_map_floor_rule_uneven():
     # floor(i*H_kv/H_q) for H_q=6, H_kv=4: group sizes 2,1,2,1 and every group is used.
     got = [oracle.group_of_head(i, 6, 4) for i in range(6)]
