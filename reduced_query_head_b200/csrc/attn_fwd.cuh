@@ -14,7 +14,8 @@
 //
 // Warp roles (12 warps):
 //   warp 0   TMA producer: Q0/Q1 once, then K_j and V_j into a ring of stages
-//   warp 1   MMA issuer: S_k = Q_k K_j^T into TMEM, O_k += P_k V_j from TMEM
+//   warps 1, 3  MMA issuers, one per query tile k: S_k = Q_k K_j^T into TMEM,
+//            O_k += P_k V_j with P_k read from TMEM
 //   warp 2   owns the TMEM allocation
 //   warps 4-7 / 8-11  softmax for tile 0 / tile 1 (thread = row = TMEM lane):
 //            online softmax with a lazily rescaled running max, P written
@@ -70,8 +71,8 @@ struct AttnCfg {
   static constexpr int BAR_P = BAR_SFREE + 2;           // [2] P_k written, O_k corrected (4 warps)
   static constexpr int BAR_PV = BAR_P + 2;              // [2] O_k += P_k V done
   static constexpr int BAR_O = BAR_PV + 2;              // [2] last PV of tile k done
-  static constexpr int BAR_DRAIN = BAR_O + 2;
-  static constexpr int N_BARS = BAR_DRAIN + 1;
+  static constexpr int BAR_DRAIN = BAR_O + 2;            // [2] per MMA thread
+  static constexpr int N_BARS = BAR_DRAIN + 2;
   static constexpr int OFF_MISC = OFF_BAR + N_BARS * 8;  // tmem base (u32), abort flag (u32)
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;  // + alignment slack
   static constexpr int THREADS = 384;
@@ -132,9 +133,12 @@ __global__ void __launch_bounds__(384, 1)
   WaitCtl ctl{abort_flag, p.status, p.timeout_ns};
 
   if (tid == 0) {
+    const uint32_t active_tiles = (n_kv[0] > 0) + (n_kv[1] > 0);
     for (int i = 0; i < C::N_BARS; ++i) {
       const bool per_warp = (i >= C::BAR_SFREE && i < C::BAR_SFREE + 2) || (i >= C::BAR_P && i < C::BAR_P + 2);
-      mbar_init(bar(i), per_warp ? 4 : 1);
+      const bool kv_empty = i >= C::BAR_KVE && i < C::BAR_KVE + C::STAGES;
+      // a K/V stage is free once every MMA thread that uses it has committed it
+      mbar_init(bar(i), per_warp ? 4 : (kv_empty && C::SEP_P) ? active_tiles : 1);
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -151,8 +155,8 @@ __global__ void __launch_bounds__(384, 1)
   // Register split: the kernel launches with REGS_LAUNCH per thread (the host
   // checks this before launching). Warpgroup 0 (producer, MMA, TMEM owner)
   // gives registers back, the two softmax warpgroups take them:
-  // 128*REGS_CTRL + 256*REGS_SOFTMAX == 384*REGS_LAUNCH.
-  static_assert(128 * C::REGS_CTRL + 256 * C::REGS_SOFTMAX == 384 * C::REGS_LAUNCH, "register split");
+  // 128*REGS_CTRL + 256*REGS_SOFTMAX <= 384*REGS_LAUNCH.
+  static_assert(128 * C::REGS_CTRL + 256 * C::REGS_SOFTMAX <= 384 * C::REGS_LAUNCH, "register split");
   if (warp < 4) regs_release<C::REGS_CTRL>();
 
   if (warp == 0) {
@@ -195,88 +199,64 @@ __global__ void __launch_bounds__(384, 1)
         mbar_wait(bar(C::BAR_VF + s), (j / C::STAGES) & 1, drain);
       }
     }
-  } else if (warp == 1) {
-    // ======================= MMA issuer
+  } else if (!C::SEP_P && warp == 1) {
+    // ======================= MMA issuer (P over S): one thread, both tiles
+    // Order per step j: PV_0(j), S_0(j+1), PV_1(j), S_1(j+1). S_k(j+1) must
+    // follow PV_k(j) because P_k lives over S_k (one thread's MMAs run in
+    // issue order); the fixed order staggers the two tiles by one S + PV.
     if (lane == 0) {
       constexpr uint32_t IDESC_S = idesc_bf16_f32(C::BM, C::BN, 0, 0);
       constexpr uint32_t IDESC_O = idesc_bf16_f32(C::BM, D, 0, 1);
-      const uint32_t col_s[2] = {C::COL_S0, C::COL_S1};
-      const uint32_t col_o[2] = {C::COL_O0, C::COL_O1};
-      const uint32_t col_p[2] = {C::COL_P0, C::COL_P1};
-      bool ok = mbar_wait(bar(C::BAR_Q), 0, ctl);
       auto issue_s = [&](int k, int s) {
         const uint32_t qa = sbase + C::OFF_Q + k * C::Q_BYTES;
         const uint32_t ka = sbase + C::OFF_K + s * C::KV_BYTES;
+        const uint32_t col_s = k ? C::COL_S1 : C::COL_S0;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * C::CHUNK_Q + (kk & 3) * 32;
           const uint32_t offk = (kk >> 2) * C::CHUNK_KV + (kk & 3) * 32;
-          umma_ss(tmem + col_s[k], sdesc_sw128(qa + off, 16, 1024), sdesc_sw128(ka + offk, 16, 1024), IDESC_S,
+          umma_ss(tmem + col_s, sdesc_sw128(qa + off, 16, 1024), sdesc_sw128(ka + offk, 16, 1024), IDESC_S,
                   kk > 0);
         }
       };
       auto issue_pv = [&](int k, int s, int j) {
         const uint32_t va = sbase + C::OFF_V + s * C::KV_BYTES;
+        const uint32_t col_o = k ? C::COL_O1 : C::COL_O0;
+        const uint32_t col_p = k ? C::COL_P1 : C::COL_P0;
 #pragma unroll
         for (int kk = 0; kk < C::BN / 16; ++kk) {
-          umma_ts(tmem + col_o[k], tmem + col_p[k] + kk * 8, sdesc_sw128(va + kk * 16 * 128, C::CHUNK_KV, 1024),
+          umma_ts(tmem + col_o, tmem + col_p + kk * 8, sdesc_sw128(va + kk * 16 * 128, C::CHUNK_KV, 1024),
                   IDESC_O, (j > 0 || kk > 0) ? 1u : 0u);
         }
       };
-      if (ok && n_max > 0) {
-        ok = mbar_wait(bar(C::BAR_KF + 0), 0, ctl);
-        if (ok) {
-          tc_fence_after();
-          for (int k = 0; k < 2; ++k)
-            if (n_kv[k] > 0) {
-              issue_s(k, 0);
-              umma_commit(bar(C::BAR_S + k));
-            }
-        }
+      bool ok = n_max > 0 && mbar_wait(bar(C::BAR_Q), 0, ctl) && mbar_wait(bar(C::BAR_KF + 0), 0, ctl);
+      if (ok) {
+        tc_fence_after();
+        for (int k = 0; k < 2; ++k)
+          if (n_kv[k] > 0) {
+            issue_s(k, 0);
+            umma_commit(bar(C::BAR_S + k));
+          }
       }
       for (int j = 0; ok && j < n_max; ++j) {
         const int s = j % C::STAGES;
         const uint32_t ph = (j / C::STAGES) & 1;
         const int s1 = (j + 1) % C::STAGES;
         const uint32_t ph1 = ((j + 1) / C::STAGES) & 1;
-        if constexpr (C::SEP_P) {
-          // S_k(j+1) as soon as softmax k has read S_k(j): overlaps softmax k(j).
-          for (int k = 0; k < 2 && ok; ++k) {
-            if (j + 1 >= n_kv[k]) continue;
-            if (!mbar_wait(bar(C::BAR_SFREE + k), j & 1, ctl) || !mbar_wait(bar(C::BAR_KF + s1), ph1, ctl)) {
-              ok = false;
-              break;
-            }
+        if (!mbar_wait(bar(C::BAR_VF + s), ph, ctl)) { ok = false; break; }
+        for (int k = 0; k < 2 && ok; ++k) {
+          if (j >= n_kv[k]) continue;
+          if (!mbar_wait(bar(C::BAR_P + k), j & 1, ctl)) { ok = false; break; }
+          tc_fence_after();
+          issue_pv(k, s, j);
+          umma_commit(bar(C::BAR_PV + k));
+          if (j == n_kv[k] - 1) {
+            umma_commit(bar(C::BAR_O + k));
+          } else {
+            if (!mbar_wait(bar(C::BAR_KF + s1), ph1, ctl)) { ok = false; break; }
             tc_fence_after();
             issue_s(k, s1);
             umma_commit(bar(C::BAR_S + k));
-          }
-          if (!ok || !mbar_wait(bar(C::BAR_VF + s), ph, ctl)) { ok = false; break; }
-          for (int k = 0; k < 2 && ok; ++k) {
-            if (j >= n_kv[k]) continue;
-            if (!mbar_wait(bar(C::BAR_P + k), j & 1, ctl)) { ok = false; break; }
-            tc_fence_after();
-            issue_pv(k, s, j);
-            umma_commit(bar(C::BAR_PV + k));
-            if (j == n_kv[k] - 1) umma_commit(bar(C::BAR_O + k));
-          }
-        } else {
-          // P lives over S_k: S_k(j+1) may only follow PV_k(j) (MMAs run in issue order).
-          if (!mbar_wait(bar(C::BAR_VF + s), ph, ctl)) { ok = false; break; }
-          for (int k = 0; k < 2 && ok; ++k) {
-            if (j >= n_kv[k]) continue;
-            if (!mbar_wait(bar(C::BAR_P + k), j & 1, ctl)) { ok = false; break; }
-            tc_fence_after();
-            issue_pv(k, s, j);
-            umma_commit(bar(C::BAR_PV + k));
-            if (j == n_kv[k] - 1) {
-              umma_commit(bar(C::BAR_O + k));
-            } else {
-              if (!mbar_wait(bar(C::BAR_KF + s1), ph1, ctl)) { ok = false; break; }
-              tc_fence_after();
-              issue_s(k, s1);
-              umma_commit(bar(C::BAR_S + k));
-            }
           }
         }
         umma_commit(bar(C::BAR_KVE + s));
@@ -286,6 +266,79 @@ __global__ void __launch_bounds__(384, 1)
       volatile int zero = 0;
       WaitCtl drain{&zero, p.status, p.timeout_ns};
       mbar_wait(bar(C::BAR_DRAIN), 0, drain);
+    }
+  } else if (C::SEP_P && (warp == 1 || warp == 3)) {
+    // ======================= MMA issuers (P in its own columns): one thread per tile
+    // Each tile's S/PV chain runs on its own thread, so a slow step of one
+    // tile never holds up the other (issue blocks until the tensor core
+    // accepts the MMA). Both threads feed the same tensor core; they touch
+    // disjoint TMEM columns and meet only on the K/V stage barriers.
+    const int k = warp == 1 ? 0 : 1;
+    if (lane == 0) {
+      constexpr uint32_t IDESC_S = idesc_bf16_f32(C::BM, C::BN, 0, 0);
+      constexpr uint32_t IDESC_O = idesc_bf16_f32(C::BM, D, 0, 1);
+      const uint32_t col_s = k ? C::COL_S1 : C::COL_S0;
+      const uint32_t col_o = k ? C::COL_O1 : C::COL_O0;
+      const uint32_t col_p = k ? C::COL_P1 : C::COL_P0;
+      const uint32_t qa = sbase + C::OFF_Q + k * C::Q_BYTES;
+      const int nk = n_kv[k];
+      auto issue_s = [&](int s) {
+        const uint32_t ka = sbase + C::OFF_K + s * C::KV_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * C::CHUNK_Q + (kk & 3) * 32;
+          const uint32_t offk = (kk >> 2) * C::CHUNK_KV + (kk & 3) * 32;
+          umma_ss(tmem + col_s, sdesc_sw128(qa + off, 16, 1024), sdesc_sw128(ka + offk, 16, 1024), IDESC_S,
+                  kk > 0);
+        }
+      };
+      auto issue_pv = [&](int s, int j) {
+        const uint32_t va = sbase + C::OFF_V + s * C::KV_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < C::BN / 16; ++kk) {
+          umma_ts(tmem + col_o, tmem + col_p + kk * 8, sdesc_sw128(va + kk * 16 * 128, C::CHUNK_KV, 1024),
+                  IDESC_O, (j > 0 || kk > 0) ? 1u : 0u);
+        }
+      };
+      bool ok = nk > 0 && mbar_wait(bar(C::BAR_Q), 0, ctl) && mbar_wait(bar(C::BAR_KF + 0), 0, ctl);
+      if (ok) {
+        tc_fence_after();
+        issue_s(0);
+        umma_commit(bar(C::BAR_S + k));
+      }
+      for (int j = 0; ok && j < nk; ++j) {
+        const int s = j % C::STAGES;
+        const uint32_t ph = (j / C::STAGES) & 1;
+        const int s1 = (j + 1) % C::STAGES;
+        const uint32_t ph1 = ((j + 1) / C::STAGES) & 1;
+        const bool more = j + 1 < nk;
+        {
+          // S(j+1) as soon as the softmax has read S(j): overlaps softmax(j).
+          if (more) {
+            if (!mbar_wait(bar(C::BAR_SFREE + k), j & 1, ctl) || !mbar_wait(bar(C::BAR_KF + s1), ph1, ctl)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            issue_s(s1);
+            umma_commit(bar(C::BAR_S + k));
+          }
+        }
+        if (!mbar_wait(bar(C::BAR_VF + s), ph, ctl) || !mbar_wait(bar(C::BAR_P + k), j & 1, ctl)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        issue_pv(s, j);
+        umma_commit(bar(C::BAR_PV + k));
+        if (!more) umma_commit(bar(C::BAR_O + k));
+        umma_commit(bar(C::BAR_KVE + s));
+      }
+      // Drain: every MMA issued above has finished before TMEM is released.
+      umma_commit(bar(C::BAR_DRAIN + k));
+      volatile int zero = 0;
+      WaitCtl drain{&zero, p.status, p.timeout_ns};
+      mbar_wait(bar(C::BAR_DRAIN + k), 0, drain);
     }
   } else if (warp >= 4) {
     // ======================= softmax + epilogue, one thread per tile row
