@@ -90,6 +90,38 @@ int sqa_layer_fwd(const void* x, const void* Wq, const void* Wk, const void* Wv,
                   int causal, float scale, void* stream);
 
 /*
+ * Size of the library's own per-device scratch array used by
+ * sqa_layer_fwd_static_ws (64 MiB; every device that loads the library holds
+ * it until the process exits).
+ */
+#define SQA_STATIC_WORKSPACE_BYTES (64u << 20)
+
+/*
+ * sqa_layer_fwd without a caller-provided workspace. The pages have no
+ * counterpart to this entry point; it exists for callers that cannot allocate
+ * device memory -- a framework that owns all device memory through its own
+ * allocator and budget, or a plugin interface that passes the library only
+ * input and output buffers. The caller still provides x, the weights and out;
+ * the layer's Q/K/V/attention scratch lives in one library-owned array of
+ * SQA_STATIC_WORKSPACE_BYTES per device. Nothing is allocated per call.
+ *   - Same arguments, layouts, arithmetic and results as sqa_layer_fwd.
+ *   - Returns SQA_ERR_WORKSPACE, without launching anything, when
+ *     sqa_layer_workspace_bytes(B, N, d_model, H_q, H_kv, d_head) exceeds
+ *     SQA_STATIC_WORKSPACE_BYTES (e.g. B*N*(2*H_q + 2*H_kv)*d_head*2 bytes
+ *     above 64 MiB); SQA_ERR_INVALID_ARG for sizes sqa_layer_fwd rejects.
+ *   - The first call on a device looks up the array's device address (with
+ *     that device current) and caches it; make that first call before any
+ *     stream capture.
+ *   - All calls on a device share the one array, and it keeps the previous
+ *     call's contents. Calls whose kernels overlap on the GPU (different
+ *     streams, or host threads without ordering) race on it: order them on one
+ *     stream.
+ */
+int sqa_layer_fwd_static_ws(const void* x, const void* Wq, const void* Wk, const void* Wv, const void* Wo,
+                            void* out, int B, int N, int d_model, int H_q, int H_kv, int d_head,
+                            int causal, float scale, void* stream);
+
+/*
  * Plain projection y[M, N_out] = x[M, K] W[N_out, K]^T (bf16 in, fp32
  * accumulate, bf16 out): the layer's linear step exposed on its own.
  * Requirements: M >= 1, K >= 8, K % 8 == 0, N_out >= 8, N_out % 8 == 0.

@@ -15,14 +15,17 @@ from .build import LIB as _LIB_PATH
 __all__ = [
     "SQA_OK", "SQA_ERR_INVALID_ARG", "SQA_ERR_UNSUPPORTED", "SQA_ERR_CUDA", "SQA_ERR_TIMEOUT",
     "SQA_ERR_WORKSPACE", "SqaError", "lib", "EXPORTED_SYMBOLS", "sqa_attn_fwd", "sqa_layer_fwd",
-    "sqa_layer_workspace_bytes", "sqa_linear_fwd", "sqa_device_status", "sqa_set_wait_limit_ns",
+    "sqa_layer_workspace_bytes", "sqa_layer_fwd_static_ws", "SQA_STATIC_WORKSPACE_BYTES", "sqa_linear_fwd",
+    "sqa_device_status", "sqa_set_wait_limit_ns",
     "sqa_check_wait_timeout", "sqa_status_string", "sqa_version",
 ]
 
 SQA_OK, SQA_ERR_INVALID_ARG, SQA_ERR_UNSUPPORTED, SQA_ERR_CUDA, SQA_ERR_TIMEOUT, SQA_ERR_WORKSPACE = range(6)
+SQA_STATIC_WORKSPACE_BYTES = 64 << 20   # include/sqa.h
 
 EXPORTED_SYMBOLS = (
-    "sqa_attn_fwd", "sqa_layer_workspace_bytes", "sqa_layer_fwd", "sqa_linear_fwd", "sqa_device_status",
+    "sqa_attn_fwd", "sqa_layer_workspace_bytes", "sqa_layer_fwd", "sqa_layer_fwd_static_ws", "sqa_linear_fwd",
+    "sqa_device_status",
     "sqa_set_wait_limit_ns", "sqa_check_wait_timeout", "sqa_status_string", "sqa_version",
 )
 
@@ -40,6 +43,8 @@ lib.sqa_layer_workspace_bytes.argtypes = [_i, _i, _i, _i, _i, _i]
 lib.sqa_layer_workspace_bytes.restype = _sz
 lib.sqa_layer_fwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _i, _i, _i, _i, _i, _i, _i, _f, _vp]
 lib.sqa_layer_fwd.restype = _i
+lib.sqa_layer_fwd_static_ws.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _f, _vp]
+lib.sqa_layer_fwd_static_ws.restype = _i
 lib.sqa_linear_fwd.argtypes = [_vp, _vp, _vp, _ll, _i, _i, _vp]
 lib.sqa_linear_fwd.restype = _i
 lib.sqa_device_status.argtypes = [_vp]
@@ -103,6 +108,15 @@ def sqa_layer_fwd(x, Wq, Wk, Wv, Wo, out, workspace, workspace_bytes, B, N, d_mo
                            int(workspace_bytes), B, N, d_model, H_q, H_kv, d_head, int(causal), float(scale),
                            _stream(stream))
     return _check(st, "sqa_layer_fwd", raise_on_error)
+
+
+def sqa_layer_fwd_static_ws(x, Wq, Wk, Wv, Wo, out, B, N, d_model, H_q, H_kv, d_head, causal, scale, stream=None,
+                            raise_on_error=True):
+    """The layer with the library's own scratch array instead of a caller workspace (for callers that
+    cannot allocate device memory); problems needing more than SQA_STATIC_WORKSPACE_BYTES are refused."""
+    st = lib.sqa_layer_fwd_static_ws(_ptr(x), _ptr(Wq), _ptr(Wk), _ptr(Wv), _ptr(Wo), _ptr(out), B, N, d_model,
+                                     H_q, H_kv, d_head, int(causal), float(scale), _stream(stream))
+    return _check(st, "sqa_layer_fwd_static_ws", raise_on_error)
 
 
 def sqa_linear_fwd(x, W, y, M, K, N_out, stream=None, raise_on_error=True):

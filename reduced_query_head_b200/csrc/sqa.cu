@@ -346,6 +346,51 @@ int sqa_layer_fwd(const void* x, const void* Wq, const void* Wk, const void* Wv,
   return launch_gemm(st, g2, s);
 }
 
+// ---------------------------------------------------------------------------
+// Layer forward with library-owned scratch (no allocation by anyone per call).
+//
+// Some callers cannot allocate device memory for the layer's workspace: a
+// framework that owns all device memory through its own allocator and budget,
+// or a plugin interface that hands the library only its input and output
+// buffers. For them the library keeps one fixed scratch array per device, sized
+// SQA_STATIC_WORKSPACE_BYTES, that lives from library load until process exit.
+static __device__ __align__(256) unsigned char g_sqa_static_ws[SQA_STATIC_WORKSPACE_BYTES];
+
+namespace {
+std::mutex g_static_mu;
+void* g_static_ws_ptr[kMaxDevices] = {};
+
+// Once per device, with that device current: the array's device address. In
+// host code the array's name is only a host-side stand-in, so the address must
+// come from the runtime.
+int static_workspace(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return SQA_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_static_mu);
+  if (!g_static_ws_ptr[dev]) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_sqa_static_ws) != cudaSuccess || ptr == nullptr) return SQA_ERR_CUDA;
+    g_static_ws_ptr[dev] = ptr;
+  }
+  *out = g_static_ws_ptr[dev];
+  return SQA_OK;
+}
+}  // namespace
+
+int sqa_layer_fwd_static_ws(const void* x, const void* Wq, const void* Wk, const void* Wv, const void* Wo, void* out,
+                            int B, int N, int d_model, int H_q, int H_kv, int d_head, int causal, float scale,
+                            void* stream) {
+  const size_t need = sqa_layer_workspace_bytes(B, N, d_model, H_q, H_kv, d_head);
+  if (need == 0) return SQA_ERR_INVALID_ARG;
+  if (need > (size_t)SQA_STATIC_WORKSPACE_BYTES) return SQA_ERR_WORKSPACE;  // problem too large for the array
+  void* ws = nullptr;
+  if (int e = static_workspace(&ws)) return e;
+  // Q, K, V and the attention output are written in full before they are read,
+  // so nothing in the array has to start at zero.
+  return sqa_layer_fwd(x, Wq, Wk, Wv, Wo, out, ws, (size_t)SQA_STATIC_WORKSPACE_BYTES, B, N, d_model, H_q, H_kv,
+                       d_head, causal, scale, stream);
+}
+
 int sqa_linear_fwd(const void* x, const void* W, void* y, long long M, int K, int N_out, void* stream) {
   if (!aligned16(x) || !aligned16(W) || !aligned16(y)) return SQA_ERR_INVALID_ARG;
   if (M < 1 || M > INT_MAX || K < 8 || K % 8 != 0 || N_out < 8 || N_out % 8 != 0) return SQA_ERR_INVALID_ARG;
