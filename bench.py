@@ -35,6 +35,66 @@ METRIC = "attention TFLOP/s (4*B*N^2*H_q*d, halved if causal)"
 L2_FLUSH_BYTES = 256 << 20     # > 126 MB L2
 
 
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "attn_traffic_headcfg32k.json")
+KERNEL_SOURCES = ["attn_fwd.cuh", "sm100.cuh", "sqa.cu"]
+
+
+def kernel_source_hash():
+    """sha256 over the attention kernel's sources: DRAM counters taken from an
+    older build of the kernel are not reported against a newer one."""
+    import hashlib
+    h = hashlib.sha256()
+    for name in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, "reduced_query_head_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def ingest_traffic(paths):
+    """ncu --csv exports named traffic_<H_q>_<H_kv>.csv -> the committed per-launch DRAM bytes file."""
+    import csv
+    import re
+    per = {}
+    for path in paths:
+        m = re.search(r"traffic_(\d+)_(\d+)\.csv$", path)
+        rows = list(csv.reader(open(path)))
+        hi = [i for i, r in enumerate(rows) if r and r[0] == "ID"][0]
+        h = rows[hi]
+        mi, vi, ui = h.index("Metric Name"), h.index("Metric Value"), h.index("Metric Unit")
+        unit = {"byte": 1, "Kbyte": 1e3, "Mbyte": 1e6, "Gbyte": 1e9}
+        vals = {r[mi]: float(r[vi].replace(",", "")) * unit.get(r[ui], 1) for r in rows[hi + 1:] if len(r) > vi}
+        per["%s/%s" % (m.group(1), m.group(2))] = {
+            "dram_read_bytes": vals["dram__bytes_read.sum"], "dram_write_bytes": vals["dram__bytes_write.sum"],
+            "ncu_duration_ns": vals.get("gpu__time_duration.sum")}
+    out = {"kernel_source_sha256": kernel_source_hash(), "per_config": per,
+           "command": "ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum,gpu__time_duration.sum "
+                      "--clock-control none -k regex:attn_fwd -s 1 -c 1 --csv python bench.py --workload single "
+                      "--N 32768 --hq <H_q> --hkv <H_kv> --d 64 --steps 1 --warmup 1"}
+    os.makedirs(os.path.dirname(TRAFFIC_FILE), exist_ok=True)
+    with open(TRAFFIC_FILE, "w") as f:
+        json.dump(out, f, indent=1)
+        f.write("\n")
+    return out
+
+
+def load_traffic(names_hq_hkv):
+    """Mean DRAM bytes per attention launch over the given configs, or None if
+    the counters were taken on another build of the kernel."""
+    if not os.path.exists(TRAFFIC_FILE):
+        return None, "no capture"
+    with open(TRAFFIC_FILE) as f:
+        t = json.load(f)
+    if t.get("kernel_source_sha256") != kernel_source_hash():
+        return None, "capture is from an older kernel build"
+    vals = []
+    for H_q, H_kv in names_hq_hkv:
+        e = t["per_config"].get("%d/%d" % (H_q, H_kv))
+        if e is None:
+            return None, "config missing from capture"
+        vals.append(e["dram_read_bytes"] + e["dram_write_bytes"])
+    return sum(vals) / len(vals), "ncu dram__bytes_read.sum + dram__bytes_write.sum, mean per launch"
+
+
 def attn_flops(B, N, H_q, d, causal):
     f = 4.0 * B * N * N * H_q * d
     return f / 2 if causal else f
@@ -228,6 +288,8 @@ def bench_sqa(args):
     e2e_value = flops_step * world / (e2e_ms_max * 1e-3) / 1e12
     launch_ms = step_ms / len(cfgs)
     achieved = (flops_step / len(cfgs)) / (launch_ms * 1e-3) / 1e12
+    traffic, traffic_src = load_traffic([(c["H_q"], c["H_kv"]) for c in cfgs])
+    alg_bytes = sum(2 * c["B"] * c["N"] * c["d"] * (2 * c["H_q"] + 2 * c["H_kv"]) for c in cfgs) / len(cfgs)
     peak = peaks["bf16_tflops"]
 
     result = None
@@ -255,7 +317,8 @@ def bench_sqa(args):
             "roofline": {"bound": "tensor", "kernel": "sqa::attn_fwd_kernel<64>", "achieved": round(achieved, 1),
                          "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 3),
                          "peak_source": peaks["source"] + " bf16 dense (burst; each launch timed alone)",
-                         "traffic": args.traffic},
+                         "traffic": traffic, "traffic_source": traffic_src,
+                         "algorithmic_bytes_per_launch": alg_bytes},
             "e2e": {"value": round(e2e_value, 2), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms_max, 4)},
             "gpu_launches": args.steps * len(cfgs),
@@ -482,9 +545,12 @@ def main():
     ap.add_argument("--causal", type=int, default=0)
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--traffic", type=float, default=None,
-                    help="ncu dram bytes per attention launch, if captured for this kernel build")
+    ap.add_argument("--ingest-traffic", nargs="+", default=None, metavar="CSV",
+                    help="write the per-launch DRAM traffic file from ncu CSV exports, then exit")
     args = ap.parse_args()
+    if args.ingest_traffic:
+        print(json.dumps(ingest_traffic(args.ingest_traffic)))
+        return
     if args.warmup < 3 and args.impl == "sqa" and args.workload == "headcfg32k":
         print("note: raising --warmup to 3", file=sys.stderr)
         args.warmup = 3

@@ -7,7 +7,8 @@
 // diagram); Sparse Query Attention is the same computation with fewer query
 // heads ("Sparse Query Attention (SQA)", abstract).
 //
-// One CTA owns two 128-row query tiles of one (batch, head block). A head
+// One CTA owns two 128-row query tiles of one (batch, head block), or one
+// tile when the host splits the last non-causal pairs to fill the final wave. A head
 // block is P consecutive query heads of one KV group (P a power of two
 // dividing H_q/H_kv), stacked so that tile row r = token_local * P + head
 // offset: every key/value tile brought into shared memory serves all P heads.
@@ -19,9 +20,12 @@
 //   warp 2   owns the TMEM allocation
 //   warps 4-7 / 8-11  softmax for tile 0 / tile 1 (thread = row = TMEM lane):
 //            online softmax with a lazily rescaled running max, P written
-//            back to TMEM as bf16 over S, epilogue O / l -> bf16 -> global.
+//            back to TMEM as bf16, epilogue O / l -> bf16 -> global.
+// At d=128 P is written over S, so S_k(j+1) must follow PV_k(j): one thread
+// (warp 1) issues both tiles' MMAs in the order PV_0, S_0, PV_1, S_1.
 //
-// TMEM columns: S0 [0,128), S1 [128,256), O0 [256,256+D), O1 [256+D,256+2D).
+// TMEM columns: S0 [0,128), S1 [128,256), O0 [256,256+D), O1 [256+D,256+2D);
+// P0/P1 in [384,448)/[448,512) at d=64, over S0/S1 at d=128.
 // Every wait is bounded; on time-out the kernel records the status, drains
 // its own copies and MMAs, frees TMEM and returns.
 #pragma once
@@ -36,6 +40,7 @@ struct AttnParams {
   int P, log2P;         // heads stacked per tile
   int tpt;              // tokens per 128-row tile = 128 / P
   int n_pairs;          // tile pairs per (batch, head block)
+  int n_pair_items;     // CTAs [0, n_pair_items) run two tiles; the rest run one tile each
   int n_hb;             // head blocks = H_q / P
   int causal;
   float scale_log2;     // scale * log2(e)
@@ -105,11 +110,28 @@ __global__ void __launch_bounds__(384, 1)
   const int warp = tid >> 5;
   const int lane = tid & 31;
 
-  // ---- work item (longest first when causal)
-  const int per_pair = p.n_hb * p.B;
-  int qp = blockIdx.x / per_pair;
-  const int rest = blockIdx.x - qp * per_pair;
-  if (p.causal) qp = p.n_pairs - 1 - qp;
+  // ---- work item
+  // Causal: query-tile pair outermost, longest first, so the short items fill
+  // the tail. Non-causal: all items cost the same, so the query-tile pair is
+  // innermost and CTAs running together read the same head block's K/V from L2.
+  // The last pairs of a non-causal grid may be split into one-tile CTAs so
+  // that the final wave is filled (the host decides, see n_pair_items).
+  int item = blockIdx.x, single = -1;
+  if (item >= p.n_pair_items) {
+    const int s = item - p.n_pair_items;
+    item = p.n_pair_items + (s >> 1);
+    single = s & 1;                      // which tile of the pair this CTA runs
+  }
+  int qp, rest;
+  if (p.causal) {
+    const int per_pair = p.n_hb * p.B;
+    qp = item / per_pair;
+    rest = item - qp * per_pair;
+    qp = p.n_pairs - 1 - qp;
+  } else {
+    qp = item % p.n_pairs;
+    rest = item / p.n_pairs;
+  }
   const int hb = rest % p.n_hb;
   const int b = rest / p.n_hb;
   const int head0 = hb * p.P;
@@ -119,6 +141,7 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
   for (int k = 0; k < 2; ++k) {
     t0[k] = (qp * 2 + k) * p.tpt;
+    if (single >= 0) t0[k] = (k == 0) ? (qp * 2 + single) * p.tpt : p.N;  // one tile, in slot 0
     if (t0[k] >= p.N) {
       n_kv[k] = 0;
     } else if (p.causal) {
@@ -138,7 +161,7 @@ __global__ void __launch_bounds__(384, 1)
       const bool per_warp = (i >= C::BAR_SFREE && i < C::BAR_SFREE + 2) || (i >= C::BAR_P && i < C::BAR_P + 2);
       const bool kv_empty = i >= C::BAR_KVE && i < C::BAR_KVE + C::STAGES;
       // a K/V stage is free once every MMA thread that uses it has committed it
-      mbar_init(bar(i), per_warp ? 4 : (kv_empty && C::SEP_P) ? active_tiles : 1);
+      mbar_init(bar(i), per_warp ? 4 : (kv_empty && C::SEP_P && active_tiles > 1) ? 2 : 1);
     }
     *abort_flag = 0;
     fence_mbar_init();

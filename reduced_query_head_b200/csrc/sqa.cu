@@ -161,7 +161,16 @@ int launch_attn(const DeviceState* st, const void* q, const void* k, const void*
   const int tpt = C::BM / P;
   const long long n_pairs = ((long long)N + 2 * tpt - 1) / (2 * tpt);
   const long long n_hb = H_q / P;
-  const long long grid = n_pairs * n_hb * B;
+  const long long pairs = n_pairs * n_hb * B;
+  // Non-causal items all cost the same. When the pairs left over after the
+  // full waves fit in one wave as single tiles, run them that way: the last
+  // wave then finishes sooner (its softmax warps do not share MUFU units).
+  long long pair_items = pairs, grid = pairs;
+  const long long rem = pairs % st->sms;
+  if (!causal && rem > 0 && 2 * rem <= st->sms) {
+    pair_items = pairs - rem;
+    grid = pairs + rem;
+  }
   if (grid > INT_MAX) return SQA_ERR_INVALID_ARG;
 
   CUtensorMap tq, tk, tv;
@@ -188,6 +197,7 @@ int launch_attn(const DeviceState* st, const void* q, const void* k, const void*
   p.log2P = log2P;
   p.tpt = tpt;
   p.n_pairs = (int)n_pairs;
+  p.n_pair_items = (int)pair_items;
   p.n_hb = (int)n_hb;
   p.causal = causal;
   p.scale_log2 = (float)((double)scale * 1.4426950408889634);  // scale * log2(e)
