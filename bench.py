@@ -7,12 +7,13 @@ xSMQA (4,1). One step runs sqa_attn_fwd once per head configuration; the
 metric is useful attention TFLOP/s = sum 4*B*N^2*H_q*d / device time.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl sqa|reference]
-                    [--workload headcfg32k|long|layer|sweep]
+                    [--workload headcfg32k|small|long|layer|sweep|single]
 
 `--impl reference` times the float64 CPU oracle on a bounded sample of the
 same workload (rank 0 only). Other workloads print extra measurement lines
-(not the headline): `long` = config N in {65536,131072,200000}, `layer` = the
-causal layer x[4,16384,2048], `sweep` = the d=128 cost grid.
+(not the headline): `small` = B=1 N=1024 (us and GB/s), `long` = N in
+{65536,131072,200000}, `layer` = the causal layer x[4,16384,2048], `sweep` =
+the d=128 cost grid, `single` = one configuration (for profiler captures).
 """
 from __future__ import annotations
 
@@ -471,6 +472,35 @@ def _bench_extra(args, sqa, torch, device, stream, flush, peaks, lines):
                           "pct_of_peak": round(100 * fl / (med * 1e-3) / 1e12 / peaks["bf16_tflops"], 1)})
             print(json.dumps(lines[-1]), flush=True)
             del dev, out
+    elif args.workload == "small":
+        # config 1: B=1, N=1024, H_q=8, H_kv=4, d=64, non-causal, scale 1/8 -- latency-bound
+        B, N, H_q, H_kv, d = 1, 1024, 8, 4, 64
+        _, dev = make_attn_inputs(B, N, H_q, H_kv, d, 0, 1.0, device)
+        out = torch.empty((B, N, H_q, d), dtype=torch.bfloat16, device=device)
+
+        def fn():
+            sqa.sqa_attn_fwd(dev["q"], dev["k"], dev["v"], out, B, N, H_q, H_kv, d, 0, 0.125, stream)
+        for _ in range(max(args.warmup, 3)):
+            fn()
+        cold = _time_launches(fn, args.steps, flush, stream)
+        warm_ev = []
+        for _ in range(args.steps):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fn()
+            b.record(stream)
+            warm_ev.append((a, b))
+        torch.cuda.synchronize()
+        warm = [a.elapsed_time(b) for a, b in warm_ev]
+        assert sqa.sqa_device_status(stream) == 0
+        nbytes = 2 * B * N * d * (2 * H_q + 2 * H_kv)
+        fl = attn_flops(B, N, H_q, d, False)
+        for name, ms in (("l2_flushed", cold), ("l2_warm", warm)):
+            med = statistics.median(ms)
+            lines.append({"workload": "small", "timing": name, "us_median": round(med * 1e3, 2),
+                          "us_min": round(min(ms) * 1e3, 2), "GB_per_s": round(nbytes / (med * 1e-3) / 1e9, 1),
+                          "tflops": round(fl / (med * 1e-3) / 1e12, 1), "bytes": nbytes})
+            print(json.dumps(lines[-1]), flush=True)
     elif args.workload == "single":
         # one attention configuration, e.g. for a profiler capture
         N, H_q, H_kv, d, causal = args.N, args.hq, args.hkv, args.d, args.causal
@@ -537,7 +567,8 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["sqa", "reference"], default="sqa")
-    ap.add_argument("--workload", choices=["headcfg32k", "long", "layer", "sweep", "single"], default="headcfg32k")
+    ap.add_argument("--workload", choices=["headcfg32k", "small", "long", "layer", "sweep", "single"],
+                    default="headcfg32k")
     ap.add_argument("--N", type=int, default=32768)
     ap.add_argument("--hq", type=int, default=16)
     ap.add_argument("--hkv", type=int, default=16)
