@@ -214,7 +214,7 @@ __global__ void __launch_bounds__(384, 1)
       }
       // Drain: wait (bounded) for the copies this thread issued, so none lands after exit.
       volatile int zero = 0;
-      WaitCtl drain{&zero, p.status, p.timeout_ns};
+      WaitCtl drain{&zero, p.status, drain_limit_ns(p.timeout_ns)};
       mbar_wait(bar(C::BAR_Q), 0, drain);
       for (int j = max(0, filled - C::STAGES); j < filled; ++j) {
         const int s = j % C::STAGES;
@@ -287,7 +287,7 @@ __global__ void __launch_bounds__(384, 1)
       // Drain: every MMA issued above has finished before TMEM is released.
       umma_commit(bar(C::BAR_DRAIN));
       volatile int zero = 0;
-      WaitCtl drain{&zero, p.status, p.timeout_ns};
+      WaitCtl drain{&zero, p.status, drain_limit_ns(p.timeout_ns)};
       mbar_wait(bar(C::BAR_DRAIN), 0, drain);
     }
   } else if (C::SEP_P && (warp == 1 || warp == 3)) {
@@ -360,7 +360,7 @@ __global__ void __launch_bounds__(384, 1)
       // Drain: every MMA issued above has finished before TMEM is released.
       umma_commit(bar(C::BAR_DRAIN + k));
       volatile int zero = 0;
-      WaitCtl drain{&zero, p.status, p.timeout_ns};
+      WaitCtl drain{&zero, p.status, drain_limit_ns(p.timeout_ns)};
       mbar_wait(bar(C::BAR_DRAIN + k), 0, drain);
     }
   } else if (warp >= 4) {

@@ -112,7 +112,7 @@ __global__ void __launch_bounds__(192, 1)
       }
       // drain the copies in flight
       volatile int zero = 0;
-      WaitCtl drain{&zero, p.status, p.timeout_ns};
+      WaitCtl drain{&zero, p.status, drain_limit_ns(p.timeout_ns)};
       for (int j = max(0, it - C::STAGES); j < it; ++j)
         mbar_wait(bar(C::BAR_FULL + j % C::STAGES), (j / C::STAGES) & 1, drain);
     }
@@ -143,7 +143,7 @@ __global__ void __launch_bounds__(192, 1)
       }
       umma_commit(bar(C::BAR_DRAIN));
       volatile int zero = 0;
-      WaitCtl drain{&zero, p.status, p.timeout_ns};
+      WaitCtl drain{&zero, p.status, drain_limit_ns(p.timeout_ns)};
       mbar_wait(bar(C::BAR_DRAIN), 0, drain);
     }
   } else {

@@ -78,6 +78,13 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const W
   }
 }
 
+// Limit for the waits that drain a kernel's own copies and MMAs before it
+// releases shared memory and TMEM: never shorter than 1 s, whatever limit the
+// caller set for ordinary waits, so an early abort cannot cut a drain short.
+__device__ __forceinline__ uint64_t drain_limit_ns(uint64_t wait_limit_ns) {
+  return wait_limit_ns > 1000000000ull ? wait_limit_ns : 1000000000ull;
+}
+
 // Warp-uniform version: every lane waits, then the warp agrees on the outcome.
 __device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity, const WaitCtl& c) {
   bool ok = mbar_wait(bar, parity, c);
