@@ -501,6 +501,30 @@ def _bench_extra(args, sqa, torch, device, stream, flush, peaks, lines):
                           "us_min": round(min(ms) * 1e3, 2), "GB_per_s": round(nbytes / (med * 1e-3) / 1e9, 1),
                           "tflops": round(fl / (med * 1e-3) / 1e12, 1), "bytes": nbytes})
             print(json.dumps(lines[-1]), flush=True)
+    elif args.workload == "linear":
+        # one projection GEMM y[M, N_out] = x[M, K] W^T (default: the layer's QKV shape)
+        import synth
+        M, K, N_out = args.M, args.K, args.N_out
+
+        def mk(shape, name, factor):
+            h = torch.empty(shape, dtype=torch.bfloat16)
+            synth.fill_bf16_into(h.data_ptr(), h.numel(), 0, name, factor)
+            return h.to(device)
+        x, w = mk((M, K), "x", 1.0), mk((N_out, K), "wq", 0.02)
+        y = torch.empty((M, N_out), dtype=torch.bfloat16, device=device)
+
+        def fn():
+            sqa.sqa_linear_fwd(x, w, y, M, K, N_out, stream)
+        for _ in range(args.warmup):
+            fn()
+        ms = _time_launches(fn, args.steps, flush, stream)
+        assert sqa.sqa_device_status(stream) == 0
+        med = statistics.median(ms)
+        fl = 2.0 * M * K * N_out
+        lines.append({"workload": "linear", "M": M, "K": K, "N_out": N_out, "ms_median": round(med, 4),
+                      "tflops": round(fl / (med * 1e-3) / 1e12, 1),
+                      "pct_of_peak": round(100 * fl / (med * 1e-3) / 1e12 / peaks["bf16_tflops"], 1)})
+        print(json.dumps(lines[-1]), flush=True)
     elif args.workload == "single":
         # one attention configuration, e.g. for a profiler capture
         N, H_q, H_kv, d, causal = args.N, args.hq, args.hkv, args.d, args.causal
@@ -567,13 +591,16 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["sqa", "reference"], default="sqa")
-    ap.add_argument("--workload", choices=["headcfg32k", "small", "long", "layer", "sweep", "single"],
+    ap.add_argument("--workload", choices=["headcfg32k", "small", "long", "layer", "sweep", "single", "linear"],
                     default="headcfg32k")
     ap.add_argument("--N", type=int, default=32768)
     ap.add_argument("--hq", type=int, default=16)
     ap.add_argument("--hkv", type=int, default=16)
     ap.add_argument("--d", type=int, default=64)
     ap.add_argument("--causal", type=int, default=0)
+    ap.add_argument("--M", type=int, default=65536)
+    ap.add_argument("--K", type=int, default=2048)
+    ap.add_argument("--N_out", type=int, default=2048)
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ingest-traffic", nargs="+", default=None, metavar="CSV",

@@ -36,7 +36,7 @@ import numpy as np
 
 __all__ = [
     "group_of_head", "repeat_kv", "widen_bf16", "bf16_round", "attention",
-    "attention_rows", "linear", "layer", "layer_rows",
+    "attention_rows", "linear", "layer", "layer_rows", "attention_lse", "attention_backward",
 ]
 
 
@@ -216,3 +216,74 @@ def layer_rows(x, wq, wk, wv, wo, rows, H_q: int, H_kv: int, d: int, causal: boo
     q_rows = rnd(linear(xf[rows], wq)).reshape(len(rows), H_q, d)
     a = rnd(attention_rows(q_rows, k, v, rows, N, causal, scale)).reshape(len(rows), H_q * d)
     return linear(a, wo)
+
+
+# ---------------------------------------------------------------------------
+# Backward pass (gradients of the attention core).
+#
+# With S = scale * Q_i K_g^T (masked keys excluded), P = softmax(S) by rows and
+# O_i = P V_g, the chain rule for a loss with upstream gradient dO_i gives, for
+# each query head i and its group g = g(i):
+#   dV_g += P^T dO_i
+#   dP    = dO_i V_g^T
+#   dS    = P * (dP - rowsum(P * dP))      (softmax Jacobian, row by row)
+#   dQ_i  = scale * dS K_g
+#   dK_g += scale * dS^T Q_i
+# A group's K and V are shared by the query heads that read it (the repetition
+# of the GQA module's expand), so their gradients are the sums over those heads.
+# ---------------------------------------------------------------------------
+
+def attention_lse(q, k, causal: bool, scale: float) -> np.ndarray:
+    """Natural-log log-sum-exp of every score row: [B, N, H_q] (float64)."""
+    q, k = (np.asarray(t, dtype=np.float64) for t in (q, k))
+    B, N, H_q, d = q.shape
+    H_kv = k.shape[2]
+    out = np.empty((B, N, H_q), dtype=np.float64)
+    keys = np.arange(N)
+    for b in range(B):
+        for i in range(H_q):
+            kh = np.array(k[b, :, group_of_head(i, H_q, H_kv), :])
+            s = scale * (q[b, :, i, :] @ kh.T)
+            if causal:
+                s[keys[None, :] > keys[:, None]] = -np.inf
+            m = np.max(s, axis=1)
+            out[b, :, i] = m + np.log(np.sum(np.exp(s - m[:, None]), axis=1))
+    return out
+
+
+def _head_backward(qh, kh, vh, doh, causal, scale):
+    """Gradients for one query head against its group's K/V (all float64)."""
+    N = kh.shape[0]
+    s = scale * (qh @ kh.T)
+    if causal:
+        keys = np.arange(N)
+        s[keys[None, :] > keys[:, None]] = -np.inf
+    m = np.max(s, axis=1, keepdims=True)
+    e = np.exp(s - m)
+    p = e / np.sum(e, axis=1, keepdims=True)
+    dv = p.T @ doh
+    dp = doh @ vh.T
+    ds = p * (dp - np.sum(p * dp, axis=1, keepdims=True))
+    dq = scale * (ds @ kh)
+    dk = scale * (ds.T @ qh)
+    return dq, dk, dv
+
+
+def attention_backward(q, k, v, dout, causal: bool, scale: float):
+    """(dq [B,N,H_q,d], dk [B,N,H_kv,d], dv [B,N,H_kv,d]) for upstream gradient dout [B,N,H_q,d]."""
+    q, k, v, dout = (np.asarray(t, dtype=np.float64) for t in (q, k, v, dout))
+    B, N, H_q, d = q.shape
+    H_kv = k.shape[2]
+    dq = np.zeros_like(q)
+    dk = np.zeros_like(k)
+    dv = np.zeros_like(v)
+    for b in range(B):
+        for i in range(H_q):
+            g = group_of_head(i, H_q, H_kv)
+            kh = np.array(k[b, :, g, :])      # explicit repetition: head i's own copy
+            vh = np.array(v[b, :, g, :])
+            dqi, dki, dvi = _head_backward(q[b, :, i, :], kh, vh, dout[b, :, i, :], causal, scale)
+            dq[b, :, i, :] = dqi
+            dk[b, :, g, :] += dki               # a shared group collects every head's gradient
+            dv[b, :, g, :] += dvi
+    return dq, dk, dv
