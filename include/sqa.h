@@ -62,6 +62,51 @@ int sqa_attn_fwd(const void* q, const void* k, const void* v, void* out,
                  int causal, float scale, void* stream);
 
 /*
+ * sqa_attn_fwd that also writes the row log-sum-exp the backward pass needs:
+ *   lse [B, H_q, N] fp32, DEVICE, 16-byte aligned, written in full:
+ *   lse[b,i,t] = ln sum_u exp(scale * q[b,t,i,:] . k[b,u,g(i),:]) over the
+ *   same keys as the forward. Other arguments, requirements and results as
+ *   sqa_attn_fwd.
+ */
+int sqa_attn_fwd_lse(const void* q, const void* k, const void* v, void* out, float* lse,
+                     int B, int N, int H_q, int H_kv, int d_head,
+                     int causal, float scale, void* stream);
+
+/*
+ * Bytes of device workspace sqa_attn_bwd needs (two fp32 [B, H_q] x N row
+ * arrays, rows padded to a multiple of 4 floats). Returns 0 for invalid sizes.
+ */
+size_t sqa_attn_bwd_workspace_bytes(int B, int N, int H_q);
+
+/*
+ * Attention backward: the gradients of sum(out * dout) with respect to q, k
+ * and v, the training-time pass of the attention core (Sparse Query Attention
+ * targets pre-training and fine-tuning: "Sparse Query Attention (SQA)",
+ * abstract). With P = softmax(scale * q_i k_g^T) and
+ * D[t] = sum_c dout[t,c] * out[t,c]:
+ *   dq_i = scale * (P * (dout_i v_g^T - D)) k_g
+ *   dk_g = scale * sum over heads i of group g of (P * (dout_i v_g^T - D))^T q_i
+ *   dv_g = sum over heads i of group g of P^T dout_i
+ * so every query head adds its share to its group's key/value gradient.
+ *   q, k, v, out  as sqa_attn_fwd (out = that call's result for q, k, v)
+ *   dout [B, N, H_q, d_head] bf16 upstream gradient
+ *   lse  [B, H_q, N] fp32 from sqa_attn_fwd_lse on the same q, k, causal, scale
+ *   dq   [B, N, H_q, d_head]  bf16, written in full
+ *   dk, dv [B, N, H_kv, d_head] bf16, written in full (no accumulation into
+ *        what they held)
+ *   workspace: device memory of at least sqa_attn_bwd_workspace_bytes(B, N,
+ *        H_q), 256-byte aligned; scratch, overwritten.
+ * Requirements as sqa_attn_fwd. Arithmetic: P recomputed in fp32 from lse,
+ * P and dS rounded to bf16 as tensor-core operands, fp32 accumulation.
+ * SQA_ERR_WORKSPACE for a missing, misaligned or short workspace.
+ */
+int sqa_attn_bwd(const void* q, const void* k, const void* v, const void* out, const void* dout,
+                 const float* lse, void* dq, void* dk, void* dv,
+                 void* workspace, size_t workspace_bytes,
+                 int B, int N, int H_q, int H_kv, int d_head,
+                 int causal, float scale, void* stream);
+
+/*
  * Bytes of device workspace sqa_layer_fwd needs (Q, K, V and the merged
  * attention output, each 256-byte aligned). Returns 0 for invalid sizes.
  */

@@ -287,3 +287,104 @@ def attention_backward(q, k, v, dout, causal: bool, scale: float):
             dk[b, :, g, :] += dki               # a shared group collects every head's gradient
             dv[b, :, g, :] += dvi
     return dq, dk, dv
+
+
+def attention_backward_q_rows(q_rows, k, v, dout_rows, rows, N: int, causal: bool, scale: float,
+                              chunk: int = 32, with_bound: bool = False):
+    """dq for selected token positions only: [len(rows), H_q, d].
+
+    ``rows`` are flat positions b*N + t; ``q_rows`` and ``dout_rows`` hold the
+    query vectors and upstream gradients of exactly those positions. A query
+    row's gradient needs only its own score row, so each row follows the same
+    steps as :func:`_head_backward` (softmax, dP, the Jacobian's row sum, dS K).
+    With ``with_bound`` also returns the rows' error scales as
+    :func:`attention_backward_bound` defines them.
+    """
+    q_rows = np.asarray(q_rows, dtype=np.float64)
+    dout_rows = np.asarray(dout_rows, dtype=np.float64)
+    rows = np.asarray(rows, dtype=np.int64)
+    B, Nk, H_kv, d = k.shape
+    assert Nk == N
+    H_q = q_rows.shape[1]
+    out = np.empty((len(rows), H_q, d), dtype=np.float64)
+    bound = np.empty_like(out) if with_bound else None
+    bs, ts = rows // N, rows % N
+    keys = np.arange(N)
+
+    def one_head(b, i):
+        sel = np.nonzero(bs == b)[0]
+        g = group_of_head(i, H_q, H_kv)
+        kh = np.asarray(k[b, :, g, :], dtype=np.float64).copy()   # explicit repetition
+        vh = np.asarray(v[b, :, g, :], dtype=np.float64).copy()
+        for a in range(0, len(sel), chunk):
+            idx = sel[a:a + chunk]
+            t_idx = ts[idx]
+            n = min(N, int(t_idx.max()) + 1) if causal else N
+            s = scale * (q_rows[idx, i, :] @ kh[:n].T)
+            if causal:
+                s[keys[None, :n] > t_idx[:, None]] = -np.inf
+            m = np.max(s, axis=1, keepdims=True)
+            e = np.exp(s - m)
+            p = e / np.sum(e, axis=1, keepdims=True)
+            dp = dout_rows[idx, i, :] @ vh[:n].T
+            ds = p * (dp - np.sum(p * dp, axis=1, keepdims=True))
+            out[idx, i, :] = scale * (ds @ kh[:n])
+            if with_bound:
+                a = np.sum(np.abs(dout_rows[idx, i, :]) * (p @ np.abs(vh[:n])), axis=1, keepdims=True)
+                bound[idx, i, :] = scale * ((_U * np.abs(ds) + 2 * _U * p * a) @ np.abs(kh[:n]))
+
+    _map_pairs(one_head, [(int(b), i) for b in np.unique(bs) for i in range(H_q)])
+    return (out, bound) if with_bound else out
+
+
+# ---------------------------------------------------------------------------
+# Rounding-error scale of a bf16-operand backward (tolerance for the tests).
+#
+# A backward that feeds P and dS to bf16 matrix products with fp32 sums makes,
+# to first order, these errors (u = 2^-9, half a bf16 step, relative):
+#   P rounded:            |dP_err| <= u |P|
+#   D from a bf16 forward output O~ (|O~ - O| <= 2u sum_u P |v|, forward P and
+#   output rounding):     |D_err[t]| <= 2u A[t],  A[t] = sum_c |dO[t,c]| sum_u P[t,u] |v[u,c]|
+#   dS = P (dP - D) rounded, with that D:
+#                         |dS_err| <= u |dS| + 2u P A
+# which the products carry to
+#   dQ: scale * |dS_err| |K|,  dK: scale * |dS_err|^T |Q|,  dV: u |P|^T |dO|.
+# ---------------------------------------------------------------------------
+
+_U = 2.0 ** -9
+
+
+def _head_backward_bound(qh, kh, vh, doh, causal, scale):
+    """Error scales (eq, ek, ev) of one head's gradients, as stated above."""
+    N = kh.shape[0]
+    s = scale * (qh @ kh.T)
+    if causal:
+        keys = np.arange(N)
+        s[keys[None, :] > keys[:, None]] = -np.inf
+    m = np.max(s, axis=1, keepdims=True)
+    e = np.exp(s - m)
+    p = e / np.sum(e, axis=1, keepdims=True)
+    dp = doh @ vh.T
+    ds = p * (dp - np.sum(p * dp, axis=1, keepdims=True))
+    a = np.sum(np.abs(doh) * (p @ np.abs(vh)), axis=1, keepdims=True)
+    eds = _U * np.abs(ds) + 2 * _U * p * a
+    return scale * (eds @ np.abs(kh)), scale * (eds.T @ np.abs(qh)), _U * (p.T @ np.abs(doh))
+
+
+def attention_backward_bound(q, k, v, dout, causal: bool, scale: float):
+    """Per-element error scales (eq, ek, ev) shaped like attention_backward's results."""
+    q, k, v, dout = (np.asarray(t, dtype=np.float64) for t in (q, k, v, dout))
+    B, N, H_q, d = q.shape
+    H_kv = k.shape[2]
+    eq = np.zeros_like(q)
+    ek = np.zeros_like(k)
+    ev = np.zeros_like(v)
+    for b in range(B):
+        for i in range(H_q):
+            g = group_of_head(i, H_q, H_kv)
+            bq, bk, bv = _head_backward_bound(q[b, :, i, :], k[b, :, g, :], v[b, :, g, :], dout[b, :, i, :],
+                                              causal, scale)
+            eq[b, :, i, :] = bq
+            ek[b, :, g, :] += bk
+            ev[b, :, g, :] += bv
+    return eq, ek, ev

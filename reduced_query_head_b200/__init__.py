@@ -14,7 +14,8 @@ from .build import LIB as _LIB_PATH
 
 __all__ = [
     "SQA_OK", "SQA_ERR_INVALID_ARG", "SQA_ERR_UNSUPPORTED", "SQA_ERR_CUDA", "SQA_ERR_TIMEOUT",
-    "SQA_ERR_WORKSPACE", "SqaError", "lib", "EXPORTED_SYMBOLS", "sqa_attn_fwd", "sqa_layer_fwd",
+    "SQA_ERR_WORKSPACE", "SqaError", "lib", "EXPORTED_SYMBOLS", "sqa_attn_fwd", "sqa_attn_fwd_lse",
+    "sqa_attn_bwd_workspace_bytes", "sqa_attn_bwd", "sqa_layer_fwd",
     "sqa_layer_workspace_bytes", "sqa_layer_fwd_static_ws", "SQA_STATIC_WORKSPACE_BYTES", "sqa_linear_fwd",
     "sqa_device_status", "sqa_set_wait_limit_ns",
     "sqa_check_wait_timeout", "sqa_status_string", "sqa_version",
@@ -24,7 +25,7 @@ SQA_OK, SQA_ERR_INVALID_ARG, SQA_ERR_UNSUPPORTED, SQA_ERR_CUDA, SQA_ERR_TIMEOUT,
 SQA_STATIC_WORKSPACE_BYTES = 64 << 20   # include/sqa.h
 
 EXPORTED_SYMBOLS = (
-    "sqa_attn_fwd", "sqa_layer_workspace_bytes", "sqa_layer_fwd", "sqa_layer_fwd_static_ws", "sqa_linear_fwd",
+    "sqa_attn_fwd", "sqa_attn_fwd_lse", "sqa_attn_bwd_workspace_bytes", "sqa_attn_bwd", "sqa_layer_workspace_bytes", "sqa_layer_fwd", "sqa_layer_fwd_static_ws", "sqa_linear_fwd",
     "sqa_device_status",
     "sqa_set_wait_limit_ns", "sqa_check_wait_timeout", "sqa_status_string", "sqa_version",
 )
@@ -39,6 +40,12 @@ _vp, _i, _f, _sz, _ll, _ull = (ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ct
                                ctypes.c_longlong, ctypes.c_ulonglong)
 lib.sqa_attn_fwd.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _vp]
 lib.sqa_attn_fwd.restype = _i
+lib.sqa_attn_fwd_lse.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _vp]
+lib.sqa_attn_fwd_lse.restype = _i
+lib.sqa_attn_bwd_workspace_bytes.argtypes = [_i, _i, _i]
+lib.sqa_attn_bwd_workspace_bytes.restype = _sz
+lib.sqa_attn_bwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _i, _i, _i, _i, _i, _i, _f, _vp]
+lib.sqa_attn_bwd.restype = _i
 lib.sqa_layer_workspace_bytes.argtypes = [_i, _i, _i, _i, _i, _i]
 lib.sqa_layer_workspace_bytes.restype = _sz
 lib.sqa_layer_fwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _i, _i, _i, _i, _i, _i, _i, _f, _vp]
@@ -96,6 +103,26 @@ def sqa_attn_fwd(q, k, v, out, B, N, H_q, H_kv, d_head, causal, scale, stream=No
     st = lib.sqa_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), B, N, H_q, H_kv, d_head, int(causal),
                           float(scale), _stream(stream))
     return _check(st, "sqa_attn_fwd", raise_on_error)
+
+
+def sqa_attn_fwd_lse(q, k, v, out, lse, B, N, H_q, H_kv, d_head, causal, scale, stream=None, raise_on_error=True):
+    """sqa_attn_fwd that also writes lse [B, H_q, N] fp32 (natural-log row log-sum-exp)."""
+    st = lib.sqa_attn_fwd_lse(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, N, H_q, H_kv, d_head,
+                              int(causal), float(scale), _stream(stream))
+    return _check(st, "sqa_attn_fwd_lse", raise_on_error)
+
+
+def sqa_attn_bwd_workspace_bytes(B, N, H_q):
+    return int(lib.sqa_attn_bwd_workspace_bytes(B, N, H_q))
+
+
+def sqa_attn_bwd(q, k, v, out, dout, lse, dq, dk, dv, workspace, workspace_bytes, B, N, H_q, H_kv, d_head, causal,
+                 scale, stream=None, raise_on_error=True):
+    """Gradients dq [B,N,H_q,d], dk/dv [B,N,H_kv,d] (group-summed) of sum(out * dout)."""
+    st = lib.sqa_attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(dout), _ptr(lse), _ptr(dq), _ptr(dk),
+                          _ptr(dv), _ptr(workspace), int(workspace_bytes), B, N, H_q, H_kv, d_head, int(causal),
+                          float(scale), _stream(stream))
+    return _check(st, "sqa_attn_bwd", raise_on_error)
 
 
 def sqa_layer_workspace_bytes(B, N, d_model, H_q, H_kv, d_head):

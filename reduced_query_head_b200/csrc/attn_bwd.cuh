@@ -1,0 +1,519 @@
+// Backward pass of decoupled-head attention on sm_100a.
+//
+// With S = scale * Q_i K_g^T, P = softmax(S) and O_i = P V_g (query head i,
+// group g = floor(i * H_kv / H_q)), an upstream gradient dO_i gives
+//   dP = dO_i V_g^T,  dS = P * (dP - D),  D = rowsum(dO_i * O_i)
+//   dQ_i = scale * dS K_g,  dK_g += scale * dS^T Q_i,  dV_g += P^T dO_i.
+// The sums over i make the K/V gradients group-aware: every query head that
+// reads a group adds its share (the repetition of the GQA explainer's module,
+// "PyTorchでのGQA実装", expand). P is recomputed from the forward's row
+// log-sum-exp instead of being stored.
+//
+// Three kernels:
+//   bwd_prep   D and the log-sum-exp in log2 units, laid out [B, H_q, N]
+//   bwd_dkdv   one CTA per (128-key tile, group, batch); loops over the group's
+//              heads and the query tiles, accumulating dK and dV in TMEM
+//   bwd_dq     one CTA per 128-row query tile (heads of a group stacked as in
+//              the forward); loops over the key tiles, accumulating dQ in TMEM
+// Both main kernels keep S^T/S and dP^T/dP in TMEM and write P^T/dS^T (dS) back
+// over them as bf16, so the second-stage MMAs read their A operand from TMEM.
+#pragma once
+
+#include "sm100.cuh"
+
+namespace sqa {
+
+// ---------------------------------------------------------------- prep
+// One warp per row (b, t, i): D = sum_c dO * O (fp32), lse2 = lse * log2(e).
+// Both outputs are [B * H_q] rows of `ld` >= N floats (ld a multiple of 4, so
+// that the rows can be TMA-loaded); columns >= N are never written.
+template <int D>
+__global__ void __launch_bounds__(256) bwd_prep_kernel(const __nv_bfloat16* __restrict__ out,
+                                                       const __nv_bfloat16* __restrict__ dout,
+                                                       const float* __restrict__ lse, float* __restrict__ dsum,
+                                                       float* __restrict__ lse2, int B, int N, int H_q, int ld) {
+  const long long rows = (long long)B * N * H_q;
+  const long long row = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= rows) return;
+  constexpr int PER = D / 32;  // 2 or 4 elements per lane
+  const __nv_bfloat16* o = out + row * D + lane * PER;
+  const __nv_bfloat16* g = dout + row * D + lane * PER;
+  float acc = 0.f;
+#pragma unroll
+  for (int u = 0; u < PER; ++u) acc = fmaf(__bfloat162float(o[u]), __bfloat162float(g[u]), acc);
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+  if (lane == 0) {
+    // row = (b * N + t) * H_q + i  ->  [b, i, t]
+    const long long i = row % H_q;
+    const long long bt = row / H_q;
+    const long long t = bt % N, b = bt / N;
+    dsum[(b * H_q + i) * ld + t] = acc;
+    lse2[(b * H_q + i) * ld + t] = lse[(b * H_q + i) * N + t] * 1.4426950408889634f;
+  }
+}
+
+struct BwdParams {
+  __nv_bfloat16* dq;    // [B, N, H_q, D]
+  __nv_bfloat16* dk;    // [B, N, H_kv, D]
+  __nv_bfloat16* dv;    // [B, N, H_kv, D]
+  const float* lse2;    // [B, H_q] rows of ld: log-sum-exp in log2 units
+  const float* dsum;    // [B, H_q] rows of ld: rowsum(dO * O)
+  int ld;               // row stride of lse2 / dsum
+  int B, N, H_q, H_kv;
+  int P, log2P, tpt;    // dq kernel: heads stacked per tile, tokens per tile
+  int n_hb;             // dq kernel: head blocks = H_q / P
+  int causal;
+  float scale;          // softmax scale
+  float scale_log2;     // scale * log2(e)
+  int* status;
+  unsigned long long timeout_ns;
+};
+
+// ---------------------------------------------------------------- dK, dV
+template <int D>
+struct DkdvCfg {
+  static constexpr int KCH = D / 64;                  // 128-byte column chunks
+  static constexpr int STAGES = (D == 64) ? 4 : 2;
+  static constexpr int T_BYTES = 128 * D * 2;         // one 128-row bf16 tile
+  static constexpr int CHUNK = 128 * 128;             // bytes per column chunk of a tile
+  static constexpr int VEC_BYTES = 128 * 4;           // 128 fp32 (lse2 or dsum of a query tile)
+  static constexpr int STAGE_BYTES = 2 * T_BYTES + 2 * VEC_BYTES;  // Q_t, dO_t, lse2_t, dsum_t
+  static constexpr int OFF_K = 0, OFF_V = T_BYTES, OFF_STAGE = 2 * T_BYTES;
+  static constexpr int OFF_BAR = OFF_STAGE + STAGES * STAGE_BYTES;
+  static constexpr int BAR_KV = 0, BAR_FULL = 1, BAR_EMPTY = 1 + STAGES, BAR_S = 1 + 2 * STAGES,
+                       BAR_P = BAR_S + 1, BAR_DONE = BAR_P + 1, BAR_DRAIN = BAR_DONE + 1, N_BARS = BAR_DRAIN + 1;
+  static constexpr int OFF_MISC = OFF_BAR + N_BARS * 8;
+  static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
+  static constexpr int THREADS = 256;
+  static constexpr uint32_t TMEM_COLS = 512;
+  static constexpr uint32_t COL_S = 0, COL_DP = 128, COL_DV = 256, COL_DK = 256 + D;
+  static_assert(STAGE_BYTES % 1024 == 0, "stage alignment");
+};
+
+// Warps: 0 TMA producer, 1 MMA issuer + TMEM owner, 4-7 elementwise (thread =
+// key row = TMEM lane). TMEM: S^T [keys x queries] in [0,128), dP^T in
+// [128,256); P^T and dS^T (bf16) are written over their first 64 columns and
+// read back as the A operands of dV += P^T dO and dK += dS^T Q.
+template <int D>
+__global__ void __launch_bounds__(256, 1)
+    bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
+                    const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                    const __grid_constant__ CUtensorMap tm_lse2, const __grid_constant__ CUtensorMap tm_dsum,
+                    const BwdParams p) {
+  using C = DkdvCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+  uint32_t* misc = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
+  volatile uint32_t* tmem_slot = misc;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 1);
+  auto bar = [&](int i) { return smem_u32(&bars[i]); };
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+  // ---- work item: (key tile u, group g, batch b); causal: longest (small u) first
+  const int n_kt = (p.N + 127) / 128;
+  const int L = blockIdx.x;
+  int u, rest;
+  if (p.causal) {
+    u = L / (p.B * p.H_kv);
+    rest = L - u * (p.B * p.H_kv);
+  } else {
+    u = L % n_kt;
+    rest = L / n_kt;
+  }
+  const int g = rest % p.H_kv, b = rest / p.H_kv;
+  // query heads of group g under g(i) = floor(i * H_kv / H_q)
+  const int i0 = (int)(((long long)g * p.H_q + p.H_kv - 1) / p.H_kv);
+  const int i1 = (int)(((long long)(g + 1) * p.H_q + p.H_kv - 1) / p.H_kv);
+  const int t_start = p.causal ? u : 0;
+  const int n_qt = n_kt;
+  const int per_head = n_qt - t_start;
+  const int n_steps = (i1 - i0) * per_head;
+
+  WaitCtl ctl{abort_flag, p.status, p.timeout_ns};
+  if (tid == 0) {
+    for (int i = 0; i < C::N_BARS; ++i) mbar_init(bar(i), i == C::BAR_P ? 4 : 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32((const void*)tmem_slot), C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      mbar_arrive_expect_tx(bar(C::BAR_KV), 2 * C::T_BYTES);
+#pragma unroll
+      for (int c = 0; c < C::KCH; ++c) {
+        tma_load_4d(sbase + C::OFF_K + c * C::CHUNK, &tm_k, bar(C::BAR_KV), c * 64, g, u * 128, b);
+        tma_load_4d(sbase + C::OFF_V + c * C::CHUNK, &tm_v, bar(C::BAR_KV), c * 64, g, u * 128, b);
+      }
+      int filled = 0;
+      for (int s = 0; s < n_steps; ++s) {
+        const int st = s % C::STAGES, round = s / C::STAGES;
+        if (round > 0 && !mbar_wait(bar(C::BAR_EMPTY + st), (round - 1) & 1, ctl)) break;
+        const int i = i0 + s / per_head, t = t_start + s % per_head;
+        const uint32_t dst = sbase + C::OFF_STAGE + st * C::STAGE_BYTES;
+        mbar_arrive_expect_tx(bar(C::BAR_FULL + st), C::STAGE_BYTES);
+#pragma unroll
+        for (int c = 0; c < C::KCH; ++c) {
+          tma_load_4d(dst + c * C::CHUNK, &tm_q, bar(C::BAR_FULL + st), c * 64, i, t * 128, b);
+          tma_load_4d(dst + C::T_BYTES + c * C::CHUNK, &tm_do, bar(C::BAR_FULL + st), c * 64, i, t * 128, b);
+        }
+        tma_load_2d(dst + 2 * C::T_BYTES, &tm_lse2, bar(C::BAR_FULL + st), t * 128, b * p.H_q + i);
+        tma_load_2d(dst + 2 * C::T_BYTES + C::VEC_BYTES, &tm_dsum, bar(C::BAR_FULL + st), t * 128, b * p.H_q + i);
+        filled = s + 1;
+      }
+      volatile int zero = 0;
+      WaitCtl drain{&zero, p.status, drain_limit_ns(p.timeout_ns)};
+      mbar_wait(bar(C::BAR_KV), 0, drain);
+      for (int s = max(0, filled - C::STAGES); s < filled; ++s)
+        mbar_wait(bar(C::BAR_FULL + s % C::STAGES), (s / C::STAGES) & 1, drain);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t IDESC_S = idesc_bf16_f32(128, 128, 0, 0);
+      constexpr uint32_t IDESC_G = idesc_bf16_f32(128, D, 0, 1);
+      bool ok = mbar_wait(bar(C::BAR_KV), 0, ctl);
+      for (int s = 0; ok && s < n_steps; ++s) {
+        const int st = s % C::STAGES;
+        if (!mbar_wait(bar(C::BAR_FULL + st), (s / C::STAGES) & 1, ctl)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t qa = sbase + C::OFF_STAGE + st * C::STAGE_BYTES;
+        const uint32_t da = qa + C::T_BYTES;
+        const uint32_t ka = sbase + C::OFF_K, va = sbase + C::OFF_V;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * C::CHUNK + (kk & 3) * 32;
+          // S^T = K Q^T and dP^T = V dO^T (keys x queries)
+          umma_ss(tmem + C::COL_S, sdesc_sw128(ka + off, 16, 1024), sdesc_sw128(qa + off, 16, 1024), IDESC_S, kk > 0);
+          umma_ss(tmem + C::COL_DP, sdesc_sw128(va + off, 16, 1024), sdesc_sw128(da + off, 16, 1024), IDESC_S,
+                  kk > 0);
+        }
+        umma_commit(bar(C::BAR_S));
+        if (!mbar_wait(bar(C::BAR_P), s & 1, ctl)) { ok = false; break; }
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 128 / 16; ++kk) {
+          const uint32_t acc = (s > 0 || kk > 0) ? 1u : 0u;
+          // dV += P^T dO and dK += dS^T Q (B operands MN-major: d contiguous)
+          umma_ts(tmem + C::COL_DV, tmem + C::COL_S + kk * 8, sdesc_sw128(da + kk * 16 * 128, C::CHUNK, 1024),
+                  IDESC_G, acc);
+          umma_ts(tmem + C::COL_DK, tmem + C::COL_DP + kk * 8, sdesc_sw128(qa + kk * 16 * 128, C::CHUNK, 1024),
+                  IDESC_G, acc);
+        }
+        umma_commit(bar(C::BAR_EMPTY + st));
+      }
+      if (ok) umma_commit(bar(C::BAR_DONE));
+      umma_commit(bar(C::BAR_DRAIN));
+      volatile int zero = 0;
+      WaitCtl drain{&zero, p.status, drain_limit_ns(p.timeout_ns)};
+      mbar_wait(bar(C::BAR_DRAIN), 0, drain);
+    }
+  } else if (warp >= 4) {
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;
+    const int key = u * 128 + row;
+    const uint32_t lane_base = tmem + (uint32_t(quarter * 32) << 16);
+    const float sl2 = p.scale_log2;
+    bool ok = true;
+    for (int s = 0; s < n_steps; ++s) {
+      const int st = s % C::STAGES;
+      const int t = t_start + s % per_head;
+      if (!mbar_wait_warp(bar(C::BAR_S), s & 1, ctl) ||
+          !mbar_wait_warp(bar(C::BAR_FULL + st), (s / C::STAGES) & 1, ctl)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const float* vl = reinterpret_cast<const float*>(smem + C::OFF_STAGE + st * C::STAGE_BYTES + 2 * C::T_BYTES);
+      const float* vd = vl + 128;
+      const bool need_mask = (t * 128 + 127 >= p.N) || (p.causal && t == u) || (key >= p.N);
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t rs[32], rd[32];
+        tmem_ld32(lane_base + C::COL_S + c * 32, rs);
+        tmem_ld32(lane_base + C::COL_DP + c * 32, rd);
+        uint32_t pp[16], pd[16];
+#pragma unroll
+        for (int w = 0; w < 16; ++w) {
+          float pv[2], dv[2];
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int col = c * 32 + 2 * w + h;
+            float pe = ex2_approx(fmaf(__uint_as_float(rs[2 * w + h]), sl2, -vl[col]));
+            if (need_mask) {
+              const int q = t * 128 + col;
+              if (q >= p.N || key >= p.N || (p.causal && key > q)) pe = 0.f;
+            }
+            pv[h] = pe;
+            dv[h] = pe * (__uint_as_float(rd[2 * w + h]) - vd[col]);
+          }
+          pp[w] = pack_bf16x2(pv[0], pv[1]);
+          pd[w] = pack_bf16x2(dv[0], dv[1]);
+        }
+        // written behind the columns already read: chunk c packs into [16c, 16c+16)
+        tmem_st16(lane_base + C::COL_S + c * 16, pp);
+        tmem_st16(lane_base + C::COL_DP + c * 16, pd);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(C::BAR_P));
+    }
+    if (ok && mbar_wait_warp(bar(C::BAR_DONE), 0, ctl)) {
+      tc_fence_after();
+      const bool store = key < p.N;
+      const size_t base = (((size_t)b * p.N + (store ? key : 0)) * p.H_kv + g) * D;
+#pragma unroll
+      for (int which = 0; which < 2; ++which) {
+        __nv_bfloat16* dst = (which == 0 ? p.dv : p.dk) + base;
+        const float mul = which == 0 ? 1.0f : p.scale;
+        const uint32_t col0 = which == 0 ? C::COL_DV : C::COL_DK;
+#pragma unroll
+        for (int c = 0; c < D; c += 32) {
+          uint32_t r[32];
+          tmem_ld32(lane_base + col0 + c, r);  // all lanes: warp-collective
+          uint4 w[4];
+          uint32_t* wp = reinterpret_cast<uint32_t*>(w);
+#pragma unroll
+          for (int x = 0; x < 16; ++x)
+            wp[x] = pack_bf16x2(__uint_as_float(r[2 * x]) * mul, __uint_as_float(r[2 * x + 1]) * mul);
+          if (store) {
+            uint4* d4 = reinterpret_cast<uint4*>(dst + c);
+#pragma unroll
+            for (int x = 0; x < 4; ++x) d4[x] = w[x];
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+// ---------------------------------------------------------------- dQ
+template <int D>
+struct DqCfg {
+  static constexpr int KCH = D / 64;
+  static constexpr int STAGES = (D == 64) ? 4 : 2;
+  static constexpr int T_BYTES = 128 * D * 2;
+  static constexpr int CHUNK = 128 * 128;
+  static constexpr int STAGE_BYTES = 2 * T_BYTES;     // K_j, V_j
+  static constexpr int OFF_Q = 0, OFF_DO = T_BYTES, OFF_STAGE = 2 * T_BYTES;
+  static constexpr int OFF_BAR = OFF_STAGE + STAGES * STAGE_BYTES;
+  static constexpr int BAR_QD = 0, BAR_FULL = 1, BAR_EMPTY = 1 + STAGES, BAR_S = 1 + 2 * STAGES,
+                       BAR_P = BAR_S + 1, BAR_DONE = BAR_P + 1, BAR_DRAIN = BAR_DONE + 1, N_BARS = BAR_DRAIN + 1;
+  static constexpr int OFF_MISC = OFF_BAR + N_BARS * 8;
+  static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
+  static constexpr int THREADS = 256;
+  static constexpr uint32_t TMEM_COLS = 512;
+  static constexpr uint32_t COL_S = 0, COL_DP = 128, COL_DQ = 256;
+};
+
+// One CTA per 128-row query tile: P heads of one group stacked as in the
+// forward (row r = token_local * P + head offset), so each K/V tile serves all
+// P heads. Warps: 0 TMA, 1 MMA + TMEM owner, 4-7 elementwise (thread = row).
+template <int D>
+__global__ void __launch_bounds__(256, 1)
+    bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
+                  const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                  const BwdParams p) {
+  using C = DqCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+  uint32_t* misc = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
+  volatile uint32_t* tmem_slot = misc;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 1);
+  auto bar = [&](int i) { return smem_u32(&bars[i]); };
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+  // ---- work item (query tile qt, head block hb, batch b); causal: longest first
+  const int n_qt = (p.N + p.tpt - 1) / p.tpt;
+  const int L = blockIdx.x;
+  int qt, rest;
+  if (p.causal) {
+    qt = n_qt - 1 - L / (p.B * p.n_hb);
+    rest = L % (p.B * p.n_hb);
+  } else {
+    qt = L % n_qt;
+    rest = L / n_qt;
+  }
+  const int hb = rest % p.n_hb, b = rest / p.n_hb;
+  const int head0 = hb * p.P;
+  const int g = (int)(((long long)head0 * p.H_kv) / p.H_q);
+  const int t0 = qt * p.tpt;
+  const int t_last = min(p.N - 1, t0 + p.tpt - 1);
+  const int n_kt = (p.N + 127) / 128;
+  const int n_kv = p.causal ? (t_last / 128 + 1) : n_kt;
+
+  WaitCtl ctl{abort_flag, p.status, p.timeout_ns};
+  if (tid == 0) {
+    for (int i = 0; i < C::N_BARS; ++i) mbar_init(bar(i), i == C::BAR_P ? 4 : 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32((const void*)tmem_slot), C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      mbar_arrive_expect_tx(bar(C::BAR_QD), 2 * C::T_BYTES);
+#pragma unroll
+      for (int c = 0; c < C::KCH; ++c) {
+        tma_load_4d(sbase + C::OFF_Q + c * C::CHUNK, &tm_q, bar(C::BAR_QD), c * 64, head0, t0, b);
+        tma_load_4d(sbase + C::OFF_DO + c * C::CHUNK, &tm_do, bar(C::BAR_QD), c * 64, head0, t0, b);
+      }
+      int filled = 0;
+      for (int j = 0; j < n_kv; ++j) {
+        const int st = j % C::STAGES, round = j / C::STAGES;
+        if (round > 0 && !mbar_wait(bar(C::BAR_EMPTY + st), (round - 1) & 1, ctl)) break;
+        const uint32_t dst = sbase + C::OFF_STAGE + st * C::STAGE_BYTES;
+        mbar_arrive_expect_tx(bar(C::BAR_FULL + st), C::STAGE_BYTES);
+#pragma unroll
+        for (int c = 0; c < C::KCH; ++c) {
+          tma_load_4d(dst + c * C::CHUNK, &tm_k, bar(C::BAR_FULL + st), c * 64, g, j * 128, b);
+          tma_load_4d(dst + C::T_BYTES + c * C::CHUNK, &tm_v, bar(C::BAR_FULL + st), c * 64, g, j * 128, b);
+        }
+        filled = j + 1;
+      }
+      volatile int zero = 0;
+      WaitCtl drain{&zero, p.status, drain_limit_ns(p.timeout_ns)};
+      mbar_wait(bar(C::BAR_QD), 0, drain);
+      for (int j = max(0, filled - C::STAGES); j < filled; ++j)
+        mbar_wait(bar(C::BAR_FULL + j % C::STAGES), (j / C::STAGES) & 1, drain);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t IDESC_S = idesc_bf16_f32(128, 128, 0, 0);
+      constexpr uint32_t IDESC_G = idesc_bf16_f32(128, D, 0, 1);
+      const uint32_t qa = sbase + C::OFF_Q, da = sbase + C::OFF_DO;
+      bool ok = mbar_wait(bar(C::BAR_QD), 0, ctl);
+      for (int j = 0; ok && j < n_kv; ++j) {
+        const int st = j % C::STAGES;
+        if (!mbar_wait(bar(C::BAR_FULL + st), (j / C::STAGES) & 1, ctl)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t ka = sbase + C::OFF_STAGE + st * C::STAGE_BYTES;
+        const uint32_t va = ka + C::T_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * C::CHUNK + (kk & 3) * 32;
+          // S = Q K^T and dP = dO V^T (rows x keys)
+          umma_ss(tmem + C::COL_S, sdesc_sw128(qa + off, 16, 1024), sdesc_sw128(ka + off, 16, 1024), IDESC_S, kk > 0);
+          umma_ss(tmem + C::COL_DP, sdesc_sw128(da + off, 16, 1024), sdesc_sw128(va + off, 16, 1024), IDESC_S,
+                  kk > 0);
+        }
+        umma_commit(bar(C::BAR_S));
+        if (!mbar_wait(bar(C::BAR_P), j & 1, ctl)) { ok = false; break; }
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 128 / 16; ++kk)
+          // dQ += dS K_j (K as an MN-major B operand: d contiguous)
+          umma_ts(tmem + C::COL_DQ, tmem + C::COL_S + kk * 8, sdesc_sw128(ka + kk * 16 * 128, C::CHUNK, 1024),
+                  IDESC_G, (j > 0 || kk > 0) ? 1u : 0u);
+        umma_commit(bar(C::BAR_EMPTY + st));
+      }
+      if (ok) umma_commit(bar(C::BAR_DONE));
+      umma_commit(bar(C::BAR_DRAIN));
+      volatile int zero = 0;
+      WaitCtl drain{&zero, p.status, drain_limit_ns(p.timeout_ns)};
+      mbar_wait(bar(C::BAR_DRAIN), 0, drain);
+    }
+  } else if (warp >= 4) {
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;
+    const int token = t0 + (row >> p.log2P);
+    const int head = head0 + (row & (p.P - 1));
+    const bool row_ok = token < p.N;
+    const uint32_t lane_base = tmem + (uint32_t(quarter * 32) << 16);
+    const float sl2 = p.scale_log2;
+    float lse2_r = 0.f, dsum_r = 0.f;
+    if (row_ok) {
+      const size_t ri = ((size_t)b * p.H_q + head) * p.ld + token;
+      lse2_r = p.lse2[ri];
+      dsum_r = p.dsum[ri];
+    }
+    bool ok = true;
+    for (int j = 0; j < n_kv; ++j) {
+      if (!mbar_wait_warp(bar(C::BAR_S), j & 1, ctl)) { ok = false; break; }
+      tc_fence_after();
+      const bool need_mask = (j == n_kv - 1) || !row_ok;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t rs[32], rd[32];
+        tmem_ld32(lane_base + C::COL_S + c * 32, rs);
+        tmem_ld32(lane_base + C::COL_DP + c * 32, rd);
+        uint32_t pd[16];
+#pragma unroll
+        for (int w = 0; w < 16; ++w) {
+          float dv[2];
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int col = c * 32 + 2 * w + h;
+            float pe = ex2_approx(fmaf(__uint_as_float(rs[2 * w + h]), sl2, -lse2_r));
+            if (need_mask) {
+              const int key = j * 128 + col;
+              if (!row_ok || key >= p.N || (p.causal && key > token)) pe = 0.f;
+            }
+            dv[h] = pe * (__uint_as_float(rd[2 * w + h]) - dsum_r);
+          }
+          pd[w] = pack_bf16x2(dv[0], dv[1]);
+        }
+        tmem_st16(lane_base + C::COL_S + c * 16, pd);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(C::BAR_P));
+    }
+    if (ok && mbar_wait_warp(bar(C::BAR_DONE), 0, ctl)) {
+      tc_fence_after();
+      __nv_bfloat16* dst = p.dq + (((size_t)b * p.N + (row_ok ? token : 0)) * p.H_q + head) * D;
+#pragma unroll
+      for (int c = 0; c < D; c += 32) {
+        uint32_t r[32];
+        tmem_ld32(lane_base + C::COL_DQ + c, r);
+        uint4 w[4];
+        uint32_t* wp = reinterpret_cast<uint32_t*>(w);
+#pragma unroll
+        for (int x = 0; x < 16; ++x)
+          wp[x] = pack_bf16x2(__uint_as_float(r[2 * x]) * p.scale, __uint_as_float(r[2 * x + 1]) * p.scale);
+        if (row_ok) {
+          uint4* d4 = reinterpret_cast<uint4*>(dst + c);
+#pragma unroll
+          for (int x = 0; x < 4; ++x) d4[x] = w[x];
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+}  // namespace sqa

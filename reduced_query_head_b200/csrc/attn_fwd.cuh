@@ -44,6 +44,7 @@ struct AttnParams {
   int n_hb;             // head blocks = H_q / P
   int causal;
   float scale_log2;     // scale * log2(e)
+  float* lse;           // optional [B, H_q, N]: natural log of sum_u exp(scale q.k_u), or nullptr
   int* status;
   unsigned long long timeout_ns;
 };
@@ -474,6 +475,10 @@ __global__ void __launch_bounds__(384, 1)
       tc_fence_after();
       const float inv_l = 1.0f / l;
       const bool store = token < p.N;
+      // log-sum-exp of the row: l sums exp2(s*sl2 - m*sl2), so
+      // ln(sum_u exp(scale*s_u)) = (m*sl2 + log2(l)) * ln(2)
+      if (p.lse != nullptr && store)
+        p.lse[((size_t)b * p.H_q + head) * p.N + token] = (m * sl2 + __log2f(l)) * 0.69314718055994531f;
       __nv_bfloat16* dst = p.out + (((size_t)b * p.N + (store ? token : 0)) * p.H_q + head) * D;
 #pragma unroll
       for (int c = 0; c < D; c += 32) {

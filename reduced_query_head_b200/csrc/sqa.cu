@@ -11,6 +11,7 @@
 #include <mutex>
 
 #include "sqa.h"
+#include "attn_bwd.cuh"
 #include "attn_fwd.cuh"
 #include "gemm.cuh"
 
@@ -21,6 +22,9 @@ namespace {
 
 using sqa::AttnCfg;
 using sqa::AttnParams;
+using sqa::BwdParams;
+using sqa::DkdvCfg;
+using sqa::DqCfg;
 using sqa::GemmCfg;
 using sqa::GemmParams;
 
@@ -107,7 +111,15 @@ int device_state(DeviceState** out) {
         return SQA_ERR_UNSUPPORTED;
     }
     if (cudaFuncSetAttribute(sqa::gemm_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             GemmCfg::SMEM_BYTES) != cudaSuccess)
+                             GemmCfg::SMEM_BYTES) != cudaSuccess ||
+        cudaFuncSetAttribute(sqa::bwd_dkdv_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             DkdvCfg<64>::SMEM_BYTES) != cudaSuccess ||
+        cudaFuncSetAttribute(sqa::bwd_dkdv_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             DkdvCfg<128>::SMEM_BYTES) != cudaSuccess ||
+        cudaFuncSetAttribute(sqa::bwd_dq_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             DqCfg<64>::SMEM_BYTES) != cudaSuccess ||
+        cudaFuncSetAttribute(sqa::bwd_dq_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             DqCfg<128>::SMEM_BYTES) != cudaSuccess)
       return SQA_ERR_CUDA;
     st.ready = true;
   }
@@ -125,6 +137,19 @@ int encode_map(CUtensorMap* m, const void* base, int rank, const cuuint64_t* dim
   CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void*>(base), dims, strides,
                         box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? SQA_OK : SQA_ERR_CUDA;
+}
+
+// Tiled fp32 map over `rows` rows of `cols` floats, `ld` floats apart (ld a
+// multiple of 4); boxes of 128 x 1, no swizzle; columns >= cols read as zero.
+int encode_rows_f32(CUtensorMap* m, const float* base, long long rows, int cols, int ld) {
+  const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)ld * 4};
+  const cuuint32_t box[2] = {128, 1};
+  const cuuint32_t es[2] = {1, 1};
+  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(base), dims, strides, box, es,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? SQA_OK : SQA_ERR_CUDA;
 }
 
@@ -153,7 +178,7 @@ int heads_per_tile(int H_q, int H_kv) {
 
 template <int D>
 int launch_attn(const DeviceState* st, const void* q, const void* k, const void* v, void* out, int B, int N, int H_q,
-                int H_kv, int causal, float scale, cudaStream_t stream) {
+                int H_kv, int causal, float scale, cudaStream_t stream, float* lse = nullptr) {
   using C = AttnCfg<D>;
   const int P = heads_per_tile(H_q, H_kv);
   int log2P = 0;
@@ -203,6 +228,7 @@ int launch_attn(const DeviceState* st, const void* q, const void* k, const void*
   p.scale_log2 = (float)((double)scale * 1.4426950408889634);  // scale * log2(e)
   p.status = st->status;
   p.timeout_ns = g_wait_ns.load();
+  p.lse = lse;
   const AttnKernel kern = D == 64 ? attn_kernel_64(emu_index(D)) : attn_kernel_128(emu_index(D));
   kern<<<(unsigned)grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);
   return cudaGetLastError() == cudaSuccess ? SQA_OK : SQA_ERR_CUDA;
@@ -265,6 +291,81 @@ int launch_gemm(const DeviceState* st, const GemmOperands& g, cudaStream_t strea
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
+// lse2 / dsum rows: a multiple of 4 floats so that every row starts 16-byte aligned.
+int bwd_row_ld(int N) { return (N + 3) & ~3; }
+size_t bwd_vec_bytes(int B, int N, int H_q) { return align256((size_t)B * H_q * bwd_row_ld(N) * 4); }
+
+template <int D>
+int launch_attn_bwd(const DeviceState* st, const void* q, const void* k, const void* v, const void* out,
+                    const void* dout, const float* lse, void* dq, void* dk, void* dv, void* workspace, int B, int N,
+                    int H_q, int H_kv, int causal, float scale, cudaStream_t stream) {
+  const int P = heads_per_tile(H_q, H_kv);
+  int log2P = 0;
+  while ((1 << log2P) < P) ++log2P;
+  const int tpt = 128 / P;
+  const long long n_kt = ((long long)N + 127) / 128;
+  const long long n_qt = ((long long)N + tpt - 1) / tpt;
+  const long long n_hb = H_q / P;
+  const long long grid_kv = n_kt * H_kv * B, grid_q = n_qt * n_hb * B;
+  const long long rows = (long long)B * N * H_q;
+  if (grid_kv > INT_MAX || grid_q > INT_MAX || (rows + 7) / 8 > INT_MAX) return SQA_ERR_INVALID_ARG;
+  const int ld = bwd_row_ld(N);
+  float* lse2 = reinterpret_cast<float*>(workspace);
+  float* dsum = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(workspace) + bwd_vec_bytes(B, N, H_q));
+
+  CUtensorMap tq1, tdo1, tqP, tdoP, tk, tv, tl, td;
+  {
+    const cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)H_q, (cuuint64_t)N, (cuuint64_t)B};
+    const cuuint64_t strides[3] = {(cuuint64_t)D * 2, (cuuint64_t)H_q * D * 2, (cuuint64_t)N * H_q * D * 2};
+    const cuuint32_t box1[4] = {64, 1, 128, 1};
+    const cuuint32_t boxP[4] = {64, (cuuint32_t)P, (cuuint32_t)tpt, 1};
+    if (int e = encode_map(&tq1, q, 4, dims, strides, box1)) return e;
+    if (int e = encode_map(&tdo1, dout, 4, dims, strides, box1)) return e;
+    if (int e = encode_map(&tqP, q, 4, dims, strides, boxP)) return e;
+    if (int e = encode_map(&tdoP, dout, 4, dims, strides, boxP)) return e;
+  }
+  {
+    const cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)H_kv, (cuuint64_t)N, (cuuint64_t)B};
+    const cuuint64_t strides[3] = {(cuuint64_t)D * 2, (cuuint64_t)H_kv * D * 2, (cuuint64_t)N * H_kv * D * 2};
+    const cuuint32_t box[4] = {64, 1, 128, 1};
+    if (int e = encode_map(&tk, k, 4, dims, strides, box)) return e;
+    if (int e = encode_map(&tv, v, 4, dims, strides, box)) return e;
+  }
+  if (int e = encode_rows_f32(&tl, lse2, (long long)B * H_q, N, ld)) return e;
+  if (int e = encode_rows_f32(&td, dsum, (long long)B * H_q, N, ld)) return e;
+
+  BwdParams p;
+  p.dq = reinterpret_cast<__nv_bfloat16*>(dq);
+  p.dk = reinterpret_cast<__nv_bfloat16*>(dk);
+  p.dv = reinterpret_cast<__nv_bfloat16*>(dv);
+  p.lse2 = lse2;
+  p.dsum = dsum;
+  p.ld = ld;
+  p.B = B;
+  p.N = N;
+  p.H_q = H_q;
+  p.H_kv = H_kv;
+  p.P = P;
+  p.log2P = log2P;
+  p.tpt = tpt;
+  p.n_hb = (int)n_hb;
+  p.causal = causal;
+  p.scale = scale;
+  p.scale_log2 = (float)((double)scale * 1.4426950408889634);
+  p.status = st->status;
+  p.timeout_ns = g_wait_ns.load();
+
+  sqa::bwd_prep_kernel<D><<<(unsigned)((rows + 7) / 8), 256, 0, stream>>>(
+      reinterpret_cast<const __nv_bfloat16*>(out), reinterpret_cast<const __nv_bfloat16*>(dout), lse, dsum, lse2, B,
+      N, H_q, ld);
+  if (cudaGetLastError() != cudaSuccess) return SQA_ERR_CUDA;
+  sqa::bwd_dkdv_kernel<D><<<(unsigned)grid_kv, DkdvCfg<D>::THREADS, DkdvCfg<D>::SMEM_BYTES, stream>>>(
+      tq1, tdo1, tk, tv, tl, td, p);
+  if (cudaGetLastError() != cudaSuccess) return SQA_ERR_CUDA;
+  sqa::bwd_dq_kernel<D><<<(unsigned)grid_q, DqCfg<D>::THREADS, DqCfg<D>::SMEM_BYTES, stream>>>(tqP, tdoP, tk, tv, p);
+  return cudaGetLastError() == cudaSuccess ? SQA_OK : SQA_ERR_CUDA;
+}
+
 __global__ void wait_probe_kernel(int* status, unsigned long long ns) {
   __shared__ alignas(8) uint64_t barrier;
   __shared__ int abort_flag;
@@ -290,6 +391,40 @@ int sqa_attn_fwd(const void* q, const void* k, const void* v, void* out, int B, 
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   return d_head == 64 ? launch_attn<64>(st, q, k, v, out, B, N, H_q, H_kv, causal, scale, s)
                       : launch_attn<128>(st, q, k, v, out, B, N, H_q, H_kv, causal, scale, s);
+}
+
+int sqa_attn_fwd_lse(const void* q, const void* k, const void* v, void* out, float* lse, int B, int N, int H_q,
+                     int H_kv, int d_head, int causal, float scale, void* stream) {
+  if (int e = check_attn_args(q, k, v, out, B, N, H_q, H_kv, d_head, causal, scale)) return e;
+  if (!aligned16(lse)) return SQA_ERR_INVALID_ARG;
+  DeviceState* st = nullptr;
+  if (int e = device_state(&st)) return e;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  return d_head == 64 ? launch_attn<64>(st, q, k, v, out, B, N, H_q, H_kv, causal, scale, s, lse)
+                      : launch_attn<128>(st, q, k, v, out, B, N, H_q, H_kv, causal, scale, s, lse);
+}
+
+size_t sqa_attn_bwd_workspace_bytes(int B, int N, int H_q) {
+  if (B < 1 || N < 1 || H_q < 1) return 0;
+  return 2 * bwd_vec_bytes(B, N, H_q);
+}
+
+int sqa_attn_bwd(const void* q, const void* k, const void* v, const void* out, const void* dout, const float* lse,
+                 void* dq, void* dk, void* dv, void* workspace, size_t workspace_bytes, int B, int N, int H_q,
+                 int H_kv, int d_head, int causal, float scale, void* stream) {
+  if (int e = check_attn_args(q, k, v, out, B, N, H_q, H_kv, d_head, causal, scale)) return e;
+  if (!aligned16(dout) || !aligned16(lse) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
+    return SQA_ERR_INVALID_ARG;
+  const size_t need = sqa_attn_bwd_workspace_bytes(B, N, H_q);
+  if (workspace == nullptr || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 || workspace_bytes < need)
+    return SQA_ERR_WORKSPACE;
+  DeviceState* st = nullptr;
+  if (int e = device_state(&st)) return e;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  return d_head == 64
+             ? launch_attn_bwd<64>(st, q, k, v, out, dout, lse, dq, dk, dv, workspace, B, N, H_q, H_kv, causal, scale, s)
+             : launch_attn_bwd<128>(st, q, k, v, out, dout, lse, dq, dk, dv, workspace, B, N, H_q, H_kv, causal, scale,
+                                    s);
 }
 
 size_t sqa_layer_workspace_bytes(int B, int N, int d_model, int H_q, int H_kv, int d_head) {

@@ -6,7 +6,7 @@ SplitMix64 stream, Box-Muller normals in float64, a per-config factor, then a
 single round-to-nearest-even to bfloat16. The C source (``synth.c``) states the
 exact recipe; this file only builds and calls it.
 
-Tensor ids: Q=0, K=1, V=2, x=3, Wq=4, Wk=5, Wv=6, Wo=7.
+Tensor ids: Q=0, K=1, V=2, x=3, Wq=4, Wk=5, Wv=6, Wo=7, dO (upstream gradient)=8.
 """
 from __future__ import annotations
 
@@ -17,7 +17,7 @@ import threading
 
 import numpy as np
 
-TENSOR_IDS = {"q": 0, "k": 1, "v": 2, "x": 3, "wq": 4, "wk": 5, "wv": 6, "wo": 7}
+TENSOR_IDS = {"q": 0, "k": 1, "v": 2, "x": 3, "wq": 4, "wk": 5, "wv": 6, "wo": 7, "do": 8}
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "synth.c")

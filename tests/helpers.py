@@ -48,6 +48,24 @@ def assert_close(got, want, what="", out_rounding=False):
     return max_abs, rel
 
 
+def assert_close_bound(got, want, bound, what=""):
+    """Backward bar: per element |got - want| <= 2 * bound + 2^-8 |want| + 1e-6, where
+    ``bound`` is the oracle's first-order rounding-error scale of a bf16-operand,
+    fp32-accumulate backward (the factor 2 covers fp32 sums of up to 2^15
+    terms and the exp2 / log-sum-exp approximations; 2^-8 |want| the bf16
+    output rounding), and relative L2 <= 5e-3 as in the forward."""
+    got = np.asarray(got, dtype=np.float64)
+    want = np.asarray(want, dtype=np.float64)
+    max_abs, rel = errors(got, want)
+    assert np.all(np.isfinite(got)), "%s: non-finite output" % what
+    excess = np.abs(got - want) - (2.0 * bound + BF16_OUT_REL * np.abs(want) + 1e-6)
+    worst = float(excess.max()) if excess.size else 0.0
+    assert worst <= 0 and rel <= REL_L2_TOL, \
+        "%s: max_abs=%.3e exceeds the rounding bound by %.3e; rel_l2=%.3e (tol %.0e)" % (
+            what, max_abs, worst, rel, REL_L2_TOL)
+    return max_abs, rel
+
+
 def attn_inputs(B, N, H_q, H_kv, d, seed=0, factor=1.0, v_factor=None):
     """bf16 bit arrays q [B,N,H_q,d], k/v [B,N,H_kv,d] from the seeded generator."""
     q = synth.bf16_bits((B, N, H_q, d), seed, "q", factor)

@@ -130,3 +130,110 @@ def test_planted_missing_group_sum_is_caught(monkeypatch):
     monkeypatch.setattr(oracle, "attention_backward", wrong)
     with pytest.raises(AssertionError):
         test_backward_matches_torch_autograd(4, 2, True)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_q_rows_match_torch_autograd(causal):
+    # the row-sampled dq against PyTorch float64 autograd at a scattered subset of positions
+    B, N, H_q, H_kv, d, scale = 2, 40, 6, 2, 8, 0.35
+    q, k, v = _rand((B, N, H_q, d), 20), _rand((B, N, H_kv, d), 21), _rand((B, N, H_kv, d), 22)
+    dout = _rand((B, N, H_q, d), 23)
+    R = H_q // H_kv
+    tq = torch.from_numpy(q).permute(0, 2, 1, 3).requires_grad_()
+    o = torch.nn.functional.scaled_dot_product_attention(
+        tq, torch.from_numpy(k).permute(0, 2, 1, 3).repeat_interleave(R, dim=1),
+        torch.from_numpy(v).permute(0, 2, 1, 3).repeat_interleave(R, dim=1), is_causal=causal, scale=scale)
+    o.backward(torch.from_numpy(dout).permute(0, 2, 1, 3))
+    want = tq.grad.permute(0, 2, 1, 3).numpy().reshape(B * N, H_q, d)
+    rows = np.array([0, 1, 7, 39, 40, 41, 55, 79])
+    got = oracle.attention_backward_q_rows(q.reshape(B * N, H_q, d)[rows], k, v,
+                                           dout.reshape(B * N, H_q, d)[rows], rows, N, causal, scale, chunk=3)
+    np.testing.assert_allclose(got, want[rows], rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_gradient_column_sums(causal):
+    # Rows of P sum to 1 and rows of dS sum to 0, so for every group g
+    #   sum_u dV_g[u] = sum over the group's heads i of sum_t dO_i[t],   sum_u dK_g[u] = 0.
+    B, N, H_q, H_kv, d, scale = 1, 23, 6, 3, 5, 0.5
+    q, k, v = _rand((B, N, H_q, d), 24), _rand((B, N, H_kv, d), 25), _rand((B, N, H_kv, d), 26)
+    dout = _rand((B, N, H_q, d), 27)
+    _, dk, dv = oracle.attention_backward(q, k, v, dout, causal, scale)
+    for g in range(H_kv):
+        heads = [i for i in range(H_q) if (i * H_kv) // H_q == g]
+        np.testing.assert_allclose(dv[0, :, g, :].sum(axis=0), dout[0][:, heads, :].sum(axis=(0, 1)), atol=1e-12)
+        np.testing.assert_allclose(dk[0, :, g, :].sum(axis=0), np.zeros(d), atol=1e-12)
+
+
+# ---------------------------------------------------------------- the backward's rounding bound
+def _rounded_model(q, k, v, dout, causal, scale, drop_d=False):
+    """The backward with the roundings a bf16-operand kernel makes: P and dS rounded to bf16,
+    D taken from a bf16 forward output, outputs rounded to bf16 (float64 elsewhere)."""
+    r = oracle.bf16_round
+    B, N, H_q, d = q.shape
+    H_kv = k.shape[2]
+    dq, dk, dv = np.zeros_like(q), np.zeros_like(k), np.zeros_like(v)
+    keys = np.arange(N)
+    for b in range(B):
+        for i in range(H_q):
+            g = (i * H_kv) // H_q
+            qh, kh, vh, doh = q[b, :, i], k[b, :, g], v[b, :, g], dout[b, :, i]
+            s = scale * qh @ kh.T
+            if causal:
+                s[keys[None, :] > keys[:, None]] = -np.inf
+            p = np.exp(s - s.max(1, keepdims=True))
+            p /= p.sum(1, keepdims=True)
+            o = r(r(p) @ vh)
+            dsum = 0.0 if drop_d else np.sum(doh * o, axis=1, keepdims=True)
+            ds = r(p * (doh @ vh.T - dsum))
+            dq[b, :, i] = r(scale * ds @ kh)
+            dk[b, :, g] += scale * ds.T @ qh
+            dv[b, :, g] += r(p).T @ doh
+    return dq, r(dk), r(dv)
+
+
+def _bf16_inputs(shape, seed):
+    return oracle.bf16_round(_rand(shape, seed))
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("H_q,H_kv,N", [(4, 4, 64), (8, 2, 96), (6, 4, 50)])
+def test_rounded_model_within_bound(H_q, H_kv, N, causal):
+    from helpers import assert_close_bound
+    d, scale = 64, 0.125
+    q, k, v = _bf16_inputs((1, N, H_q, d), 30), _bf16_inputs((1, N, H_kv, d), 31), _bf16_inputs((1, N, H_kv, d), 32)
+    dout = _bf16_inputs((1, N, H_q, d), 33)
+    exact = oracle.attention_backward(q, k, v, dout, causal, scale)
+    bound = oracle.attention_backward_bound(q, k, v, dout, causal, scale)
+    model = _rounded_model(q, k, v, dout, causal, scale)
+    for name, m, e, bd in zip("qkv", model, exact, bound):
+        assert_close_bound(m, e, bd, "d" + name)
+
+
+def test_bound_catches_planted_mistakes():
+    from helpers import assert_close_bound
+    N, H_q, H_kv, d, scale = 96, 8, 2, 64, 0.125
+    q, k, v = _bf16_inputs((1, N, H_q, d), 34), _bf16_inputs((1, N, H_kv, d), 35), _bf16_inputs((1, N, H_kv, d), 36)
+    dout = _bf16_inputs((1, N, H_q, d), 37)
+    exact = oracle.attention_backward(q, k, v, dout, True, scale)
+    bound = oracle.attention_backward_bound(q, k, v, dout, True, scale)
+    dropped = _rounded_model(q, k, v, dout, True, scale, drop_d=True)
+    with pytest.raises(AssertionError):
+        assert_close_bound(dropped[0], exact[0], bound[0], "dq without D")
+    with pytest.raises(AssertionError):
+        assert_close_bound(exact[1] * 1.01, exact[1], bound[1], "dk scaled by 1.01")
+    with pytest.raises(AssertionError):   # one key tile's worth of dv missing
+        dv = exact[2].copy()
+        dv[0, 10] = 0.0
+        assert_close_bound(dv, exact[2], bound[2], "dv row dropped")
+
+
+def test_q_rows_bound_matches_full_bound():
+    N, H_q, H_kv, d, scale = 40, 4, 2, 16, 0.3
+    q, k, v, dout = _rand((1, N, H_q, d), 38), _rand((1, N, H_kv, d), 39), _rand((1, N, H_kv, d), 40), \
+        _rand((1, N, H_q, d), 41)
+    eq, _, _ = oracle.attention_backward_bound(q, k, v, dout, True, scale)
+    rows = np.array([0, 5, 17, 39])
+    _, b = oracle.attention_backward_q_rows(q[0][rows], k, v, dout[0][rows], rows, N, True, scale,
+                                            with_bound=True)
+    np.testing.assert_allclose(b, eq[0][rows], rtol=1e-12, atol=0)
