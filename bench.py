@@ -7,13 +7,15 @@ xSMQA (4,1). One step runs sqa_attn_fwd once per head configuration; the
 metric is useful attention TFLOP/s = sum 4*B*N^2*H_q*d / device time.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl sqa|reference]
-                    [--workload headcfg32k|small|long|layer|sweep|single]
+                    [--workload headcfg32k|small|long|layer|sweep|single|linear|bwd]
 
 `--impl reference` times the float64 CPU oracle on a bounded sample of the
 same workload (rank 0 only). Other workloads print extra measurement lines
 (not the headline): `small` = B=1 N=1024 (us and GB/s), `long` = N in
 {65536,131072,200000}, `layer` = the causal layer x[4,16384,2048], `sweep` =
-the d=128 cost grid, `single` = one configuration (for profiler captures).
+the d=128 cost grid, `single` = one configuration (for profiler captures),
+`linear` = one projection GEMM, `bwd` = the attention backward (dq, dk, dv)
+at the head configurations above plus a causal d=128 case.
 """
 from __future__ import annotations
 
@@ -542,6 +544,45 @@ def _bench_extra(args, sqa, torch, device, stream, flush, peaks, lines):
         lines.append({"workload": "single", "N": N, "H_q": H_q, "H_kv": H_kv, "d": d, "causal": causal,
                       "ms_median": round(med, 3), "tflops": round(fl / (med * 1e-3) / 1e12, 1)})
         print(json.dumps(lines[-1]), flush=True)
+    elif args.workload == "bwd":
+        # attention backward (dq, dk, dv) at the forward's head configurations; --hq/--hkv/--d/--causal
+        # given explicitly (hq != 16 or hkv != 16 or d != 64 or causal) time that one configuration instead
+        import synth
+        N = args.N
+        if (args.hq, args.hkv, args.d, args.causal) != (16, 16, 64, 0):
+            grid = [("single", args.hq, args.hkv, args.d, args.causal)]
+        else:
+            grid = [(n, hq, hkv, 64, 0) for n, hq, hkv in HEAD_CONFIGS_32K] + [("SQA-d128-causal", 16, 4, 128, 1)]
+        for name, H_q, H_kv, d, causal in grid:
+            _, dev = make_attn_inputs(1, N, H_q, H_kv, d, 0, 1.0, device)
+            h = torch.empty((1, N, H_q, d), dtype=torch.bfloat16)
+            synth.fill_bf16_into(h.data_ptr(), h.numel(), 0, "do", 1.0)
+            do = h.to(device)
+            out = torch.empty((1, N, H_q, d), dtype=torch.bfloat16, device=device)
+            lse = torch.empty((1, H_q, N), dtype=torch.float32, device=device)
+            sqa.sqa_attn_fwd_lse(dev["q"], dev["k"], dev["v"], out, lse, 1, N, H_q, H_kv, d, causal, d ** -0.5,
+                                 stream)
+            ws_bytes = sqa.sqa_attn_bwd_workspace_bytes(1, N, H_q)
+            ws = torch.empty(ws_bytes, dtype=torch.uint8, device=device)
+            dq = torch.empty_like(out)
+            dk = torch.empty_like(dev["k"])
+            dv = torch.empty_like(dev["v"])
+
+            def fn():
+                sqa.sqa_attn_bwd(dev["q"], dev["k"], dev["v"], out, do, lse, dq, dk, dv, ws, ws_bytes, 1, N, H_q,
+                                 H_kv, d, causal, d ** -0.5, stream)
+            for _ in range(args.warmup):
+                fn()
+            ms = _time_launches(fn, args.steps, flush, stream)
+            assert sqa.sqa_device_status(stream) == 0
+            # algorithmic backward FLOPs: five N x N x d products per query head (S, dP, dV, dK, dQ)
+            fl = 2.5 * attn_flops(1, N, H_q, d, causal)
+            med = statistics.median(ms)
+            lines.append({"workload": "bwd", "config": name, "N": N, "H_q": H_q, "H_kv": H_kv, "d": d,
+                          "causal": causal, "ms_median": round(med, 3), "tflops": round(fl / (med * 1e-3) / 1e12, 1),
+                          "pct_of_peak": round(100 * fl / (med * 1e-3) / 1e12 / peaks["bf16_tflops"], 1)})
+            print(json.dumps(lines[-1]), flush=True)
+            del dev, out, lse, ws, dq, dk, dv, do
     elif args.workload == "layer":
         import synth
         B, N, dm, H_q, H_kv, d = 4, 16384, 2048, 16, 8, 64
@@ -591,7 +632,7 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["sqa", "reference"], default="sqa")
-    ap.add_argument("--workload", choices=["headcfg32k", "small", "long", "layer", "sweep", "single", "linear"],
+    ap.add_argument("--workload", choices=["headcfg32k", "small", "long", "layer", "sweep", "single", "linear", "bwd"],
                     default="headcfg32k")
     ap.add_argument("--N", type=int, default=32768)
     ap.add_argument("--hq", type=int, default=16)

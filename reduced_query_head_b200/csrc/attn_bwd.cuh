@@ -71,33 +71,51 @@ struct BwdParams {
   unsigned long long timeout_ns;
 };
 
+
+// Both main kernels run a two-buffer pipeline over 64-column steps. TMEM
+// buffer b (b = step & 1) holds the step's scores in [128b, 128b + 64) and
+// its dP in [128b + 64, 128b + 128); the elementwise warpgroup that owns the
+// buffer writes P / dS back as bf16 over the first 32 columns of each half.
+// The MMA thread issues step s + 2's score products right after step s's
+// gradient products, so the tensor core works on one buffer while a
+// warpgroup works on the other.
+//   warp 0      TMA producer
+//   warp 1      MMA issuer + TMEM owner
+//   warps 4-7   elementwise for even steps (thread = TMEM lane = tile row)
+//   warps 8-11  elementwise for odd steps
+
 // ---------------------------------------------------------------- dK, dV
 template <int D>
 struct DkdvCfg {
-  static constexpr int KCH = D / 64;                  // 128-byte column chunks
-  static constexpr int STAGES = (D == 64) ? 4 : 2;
-  static constexpr int T_BYTES = 128 * D * 2;         // one 128-row bf16 tile
-  static constexpr int CHUNK = 128 * 128;             // bytes per column chunk of a tile
-  static constexpr int VEC_BYTES = 128 * 4;           // 128 fp32 (lse2 or dsum of a query tile)
-  static constexpr int STAGE_BYTES = 2 * T_BYTES + 2 * VEC_BYTES;  // Q_t, dO_t, lse2_t, dsum_t
-  static constexpr int OFF_K = 0, OFF_V = T_BYTES, OFF_STAGE = 2 * T_BYTES;
-  static constexpr int OFF_BAR = OFF_STAGE + STAGES * STAGE_BYTES;
+  static constexpr int KCH = D / 64;                   // 128-byte column chunks
+  static constexpr int BQ = 64;                        // queries per step
+  static constexpr int STAGES = (D == 64) ? 8 : 4;
+  static constexpr int KV_BYTES = 128 * D * 2;         // K or V tile, 128 keys
+  static constexpr int KV_CHUNK = 128 * 128;           // one column chunk of it
+  static constexpr int T_BYTES = BQ * D * 2;           // Q_j or dO_j, 64 queries
+  static constexpr int T_CHUNK = BQ * 128;
+  static constexpr int STAGE_BYTES = 2 * T_BYTES;
+  static constexpr int VEC_BYTES = BQ * 4;             // lse2 or dsum of the step's queries
+  static constexpr int OFF_K = 0, OFF_V = KV_BYTES, OFF_STAGE = 2 * KV_BYTES;
+  static constexpr int OFF_VEC = OFF_STAGE + STAGES * STAGE_BYTES;   // [STAGES][lse2 | dsum]
+  static constexpr int OFF_BAR = OFF_VEC + STAGES * 2 * VEC_BYTES;
   static constexpr int BAR_KV = 0, BAR_FULL = 1, BAR_EMPTY = 1 + STAGES, BAR_S = 1 + 2 * STAGES,
-                       BAR_P = BAR_S + 1, BAR_DONE = BAR_P + 1, BAR_DRAIN = BAR_DONE + 1, N_BARS = BAR_DRAIN + 1;
+                       BAR_P = BAR_S + 2, BAR_DONE = BAR_P + 2, BAR_DRAIN = BAR_DONE + 1, N_BARS = BAR_DRAIN + 1;
   static constexpr int OFF_MISC = OFF_BAR + N_BARS * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
-  static constexpr int THREADS = 256;
+  static constexpr int THREADS = 384;
   static constexpr uint32_t TMEM_COLS = 512;
-  static constexpr uint32_t COL_S = 0, COL_DP = 128, COL_DV = 256, COL_DK = 256 + D;
-  static_assert(STAGE_BYTES % 1024 == 0, "stage alignment");
+  static constexpr uint32_t COL_DV = 256, COL_DK = 256 + D;
+  static_assert(STAGE_BYTES % 1024 == 0 && OFF_STAGE % 1024 == 0, "tile alignment");
 };
 
-// Warps: 0 TMA producer, 1 MMA issuer + TMEM owner, 4-7 elementwise (thread =
-// key row = TMEM lane). TMEM: S^T [keys x queries] in [0,128), dP^T in
-// [128,256); P^T and dS^T (bf16) are written over their first 64 columns and
-// read back as the A operands of dV += P^T dO and dK += dS^T Q.
+// One CTA per (128-key tile u, KV group g, batch b). Steps walk the group's
+// query heads and, per head, the 64-query tiles that can see key tile u
+// (all of them, or those from 128u on when causal). Thread = key row:
+// S^T = K Q_j^T and dP^T = V dO_j^T, then dV += P^T dO_j and dK += dS^T Q_j
+// with P^T and dS^T read from TMEM.
 template <int D>
-__global__ void __launch_bounds__(256, 1)
+__global__ void __launch_bounds__(384, 1)
     bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
                     const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                     const __grid_constant__ CUtensorMap tm_lse2, const __grid_constant__ CUtensorMap tm_dsum,
@@ -113,7 +131,7 @@ __global__ void __launch_bounds__(256, 1)
   auto bar = [&](int i) { return smem_u32(&bars[i]); };
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
-  // ---- work item: (key tile u, group g, batch b); causal: longest (small u) first
+  // ---- work item: causal items run longest (small u) first
   const int n_kt = (p.N + 127) / 128;
   const int L = blockIdx.x;
   int u, rest;
@@ -128,14 +146,14 @@ __global__ void __launch_bounds__(256, 1)
   // query heads of group g under g(i) = floor(i * H_kv / H_q)
   const int i0 = (int)(((long long)g * p.H_q + p.H_kv - 1) / p.H_kv);
   const int i1 = (int)(((long long)(g + 1) * p.H_q + p.H_kv - 1) / p.H_kv);
-  const int t_start = p.causal ? u : 0;
-  const int n_qt = n_kt;
+  const int n_qt = (p.N + C::BQ - 1) / C::BQ;
+  const int t_start = p.causal ? 2 * u : 0;
   const int per_head = n_qt - t_start;
   const int n_steps = (i1 - i0) * per_head;
 
   WaitCtl ctl{abort_flag, p.status, p.timeout_ns};
   if (tid == 0) {
-    for (int i = 0; i < C::N_BARS; ++i) mbar_init(bar(i), i == C::BAR_P ? 4 : 1);
+    for (int i = 0; i < C::N_BARS; ++i) mbar_init(bar(i), (i == C::BAR_P || i == C::BAR_P + 1) ? 4 : 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -150,11 +168,11 @@ __global__ void __launch_bounds__(256, 1)
 
   if (warp == 0) {
     if (lane == 0) {
-      mbar_arrive_expect_tx(bar(C::BAR_KV), 2 * C::T_BYTES);
+      mbar_arrive_expect_tx(bar(C::BAR_KV), 2 * C::KV_BYTES);
 #pragma unroll
       for (int c = 0; c < C::KCH; ++c) {
-        tma_load_4d(sbase + C::OFF_K + c * C::CHUNK, &tm_k, bar(C::BAR_KV), c * 64, g, u * 128, b);
-        tma_load_4d(sbase + C::OFF_V + c * C::CHUNK, &tm_v, bar(C::BAR_KV), c * 64, g, u * 128, b);
+        tma_load_4d(sbase + C::OFF_K + c * C::KV_CHUNK, &tm_k, bar(C::BAR_KV), c * 64, g, u * 128, b);
+        tma_load_4d(sbase + C::OFF_V + c * C::KV_CHUNK, &tm_v, bar(C::BAR_KV), c * 64, g, u * 128, b);
       }
       int filled = 0;
       for (int s = 0; s < n_steps; ++s) {
@@ -162,14 +180,16 @@ __global__ void __launch_bounds__(256, 1)
         if (round > 0 && !mbar_wait(bar(C::BAR_EMPTY + st), (round - 1) & 1, ctl)) break;
         const int i = i0 + s / per_head, t = t_start + s % per_head;
         const uint32_t dst = sbase + C::OFF_STAGE + st * C::STAGE_BYTES;
-        mbar_arrive_expect_tx(bar(C::BAR_FULL + st), C::STAGE_BYTES);
+        const uint32_t vec = sbase + C::OFF_VEC + st * 2 * C::VEC_BYTES;
+        const uint32_t full = bar(C::BAR_FULL + st);
+        mbar_arrive_expect_tx(full, C::STAGE_BYTES + 2 * C::VEC_BYTES);
 #pragma unroll
         for (int c = 0; c < C::KCH; ++c) {
-          tma_load_4d(dst + c * C::CHUNK, &tm_q, bar(C::BAR_FULL + st), c * 64, i, t * 128, b);
-          tma_load_4d(dst + C::T_BYTES + c * C::CHUNK, &tm_do, bar(C::BAR_FULL + st), c * 64, i, t * 128, b);
+          tma_load_4d(dst + c * C::T_CHUNK, &tm_q, full, c * 64, i, t * C::BQ, b);
+          tma_load_4d(dst + C::T_BYTES + c * C::T_CHUNK, &tm_do, full, c * 64, i, t * C::BQ, b);
         }
-        tma_load_2d(dst + 2 * C::T_BYTES, &tm_lse2, bar(C::BAR_FULL + st), t * 128, b * p.H_q + i);
-        tma_load_2d(dst + 2 * C::T_BYTES + C::VEC_BYTES, &tm_dsum, bar(C::BAR_FULL + st), t * 128, b * p.H_q + i);
+        tma_load_2d(vec, &tm_lse2, full, t * C::BQ, b * p.H_q + i);
+        tma_load_2d(vec + C::VEC_BYTES, &tm_dsum, full, t * C::BQ, b * p.H_q + i);
         filled = s + 1;
       }
       volatile int zero = 0;
@@ -180,37 +200,45 @@ __global__ void __launch_bounds__(256, 1)
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      constexpr uint32_t IDESC_S = idesc_bf16_f32(128, 128, 0, 0);
+      constexpr uint32_t IDESC_S = idesc_bf16_f32(128, C::BQ, 0, 0);
       constexpr uint32_t IDESC_G = idesc_bf16_f32(128, D, 0, 1);
-      bool ok = mbar_wait(bar(C::BAR_KV), 0, ctl);
-      for (int s = 0; ok && s < n_steps; ++s) {
+      const uint32_t ka = sbase + C::OFF_K, va = sbase + C::OFF_V;
+      // S^T = K Q_s^T and dP^T = V dO_s^T into buffer s & 1
+      auto issue_scores = [&](int s) -> bool {
         const int st = s % C::STAGES;
-        if (!mbar_wait(bar(C::BAR_FULL + st), (s / C::STAGES) & 1, ctl)) { ok = false; break; }
+        if (!mbar_wait(bar(C::BAR_FULL + st), (s / C::STAGES) & 1, ctl)) return false;
         tc_fence_after();
-        const uint32_t qa = sbase + C::OFF_STAGE + st * C::STAGE_BYTES;
-        const uint32_t da = qa + C::T_BYTES;
-        const uint32_t ka = sbase + C::OFF_K, va = sbase + C::OFF_V;
+        const uint32_t qa = sbase + C::OFF_STAGE + st * C::STAGE_BYTES, da = qa + C::T_BYTES;
+        const uint32_t buf = tmem + (uint32_t)(s & 1) * 128;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * C::CHUNK + (kk & 3) * 32;
-          // S^T = K Q^T and dP^T = V dO^T (keys x queries)
-          umma_ss(tmem + C::COL_S, sdesc_sw128(ka + off, 16, 1024), sdesc_sw128(qa + off, 16, 1024), IDESC_S, kk > 0);
-          umma_ss(tmem + C::COL_DP, sdesc_sw128(va + off, 16, 1024), sdesc_sw128(da + off, 16, 1024), IDESC_S,
-                  kk > 0);
+          const uint32_t ok_ = (kk >> 2) * C::KV_CHUNK + (kk & 3) * 32;
+          const uint32_t oq = (kk >> 2) * C::T_CHUNK + (kk & 3) * 32;
+          umma_ss(buf, sdesc_sw128(ka + ok_, 16, 1024), sdesc_sw128(qa + oq, 16, 1024), IDESC_S, kk > 0);
+          umma_ss(buf + 64, sdesc_sw128(va + ok_, 16, 1024), sdesc_sw128(da + oq, 16, 1024), IDESC_S, kk > 0);
         }
-        umma_commit(bar(C::BAR_S));
-        if (!mbar_wait(bar(C::BAR_P), s & 1, ctl)) { ok = false; break; }
+        umma_commit(bar(C::BAR_S + (s & 1)));
+        return true;
+      };
+      bool ok = mbar_wait(bar(C::BAR_KV), 0, ctl);
+      if (ok) ok = issue_scores(0);
+      if (ok && n_steps > 1) ok = issue_scores(1);
+      for (int s = 0; ok && s < n_steps; ++s) {
+        if (!mbar_wait(bar(C::BAR_P + (s & 1)), (s >> 1) & 1, ctl)) { ok = false; break; }
         tc_fence_after();
+        const int st = s % C::STAGES;
+        const uint32_t qa = sbase + C::OFF_STAGE + st * C::STAGE_BYTES, da = qa + C::T_BYTES;
+        const uint32_t buf = tmem + (uint32_t)(s & 1) * 128;
 #pragma unroll
-        for (int kk = 0; kk < 128 / 16; ++kk) {
+        for (int kk = 0; kk < C::BQ / 16; ++kk) {
           const uint32_t acc = (s > 0 || kk > 0) ? 1u : 0u;
-          // dV += P^T dO and dK += dS^T Q (B operands MN-major: d contiguous)
-          umma_ts(tmem + C::COL_DV, tmem + C::COL_S + kk * 8, sdesc_sw128(da + kk * 16 * 128, C::CHUNK, 1024),
-                  IDESC_G, acc);
-          umma_ts(tmem + C::COL_DK, tmem + C::COL_DP + kk * 8, sdesc_sw128(qa + kk * 16 * 128, C::CHUNK, 1024),
-                  IDESC_G, acc);
+          // dV += P^T dO_s and dK += dS^T Q_s (B operands MN-major: d contiguous)
+          umma_ts(tmem + C::COL_DV, buf + kk * 8, sdesc_sw128(da + kk * 16 * 128, C::T_CHUNK, 1024), IDESC_G, acc);
+          umma_ts(tmem + C::COL_DK, buf + 64 + kk * 8, sdesc_sw128(qa + kk * 16 * 128, C::T_CHUNK, 1024), IDESC_G,
+                  acc);
         }
         umma_commit(bar(C::BAR_EMPTY + st));
+        if (s + 2 < n_steps) ok = issue_scores(s + 2);
       }
       if (ok) umma_commit(bar(C::BAR_DONE));
       umma_commit(bar(C::BAR_DRAIN));
@@ -219,79 +247,83 @@ __global__ void __launch_bounds__(256, 1)
       mbar_wait(bar(C::BAR_DRAIN), 0, drain);
     }
   } else if (warp >= 4) {
+    const int wg = (warp - 4) >> 2;          // 0: even steps, 1: odd steps
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
     const int key = u * 128 + row;
     const uint32_t lane_base = tmem + (uint32_t(quarter * 32) << 16);
+    const uint32_t buf = lane_base + (uint32_t)wg * 128;
     const float sl2 = p.scale_log2;
     bool ok = true;
-    for (int s = 0; s < n_steps; ++s) {
+    for (int s = wg; s < n_steps; s += 2) {
       const int st = s % C::STAGES;
       const int t = t_start + s % per_head;
-      if (!mbar_wait_warp(bar(C::BAR_S), s & 1, ctl) ||
+      if (!mbar_wait_warp(bar(C::BAR_S + wg), (s >> 1) & 1, ctl) ||
           !mbar_wait_warp(bar(C::BAR_FULL + st), (s / C::STAGES) & 1, ctl)) {
         ok = false;
         break;
       }
       tc_fence_after();
-      const float* vl = reinterpret_cast<const float*>(smem + C::OFF_STAGE + st * C::STAGE_BYTES + 2 * C::T_BYTES);
-      const float* vd = vl + 128;
-      const bool need_mask = (t * 128 + 127 >= p.N) || (p.causal && t == u) || (key >= p.N);
+      const float4* vl4 = reinterpret_cast<const float4*>(smem + C::OFF_VEC + st * 2 * C::VEC_BYTES);
+      const float4* vd4 = vl4 + C::BQ / 4;
+      // a key above a query of the step only on the two diagonal tiles; ragged ends
+      const bool need_mask = (p.causal && t < 2 * u + 2) || (t * C::BQ + C::BQ > p.N) || (key >= p.N);
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
+      for (int c = 0; c < 2; ++c) {
         uint32_t rs[32], rd[32];
-        tmem_ld32(lane_base + C::COL_S + c * 32, rs);
-        tmem_ld32(lane_base + C::COL_DP + c * 32, rd);
+        tmem_ld32x2(buf + c * 32, buf + 64 + c * 32, rs, rd);
         uint32_t pp[16], pd[16];
 #pragma unroll
-        for (int w = 0; w < 16; ++w) {
-          float pv[2], dv[2];
+        for (int w4 = 0; w4 < 8; ++w4) {
+          const float4 l4 = vl4[c * 8 + w4], d4 = vd4[c * 8 + w4];
+          const float lv[4] = {l4.x, l4.y, l4.z, l4.w}, dv_[4] = {d4.x, d4.y, d4.z, d4.w};
+          float pv[4], dsv[4];
 #pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const int col = c * 32 + 2 * w + h;
-            float pe = ex2_approx(fmaf(__uint_as_float(rs[2 * w + h]), sl2, -vl[col]));
+          for (int h = 0; h < 4; ++h) {
+            const int col = c * 32 + w4 * 4 + h;
+            float pe = ex2_approx(fmaf(__uint_as_float(rs[w4 * 4 + h]), sl2, -lv[h]));
             if (need_mask) {
-              const int q = t * 128 + col;
+              const int q = t * C::BQ + col;
               if (q >= p.N || key >= p.N || (p.causal && key > q)) pe = 0.f;
             }
             pv[h] = pe;
-            dv[h] = pe * (__uint_as_float(rd[2 * w + h]) - vd[col]);
+            dsv[h] = pe * (__uint_as_float(rd[w4 * 4 + h]) - dv_[h]);
           }
-          pp[w] = pack_bf16x2(pv[0], pv[1]);
-          pd[w] = pack_bf16x2(dv[0], dv[1]);
+          pp[w4 * 2] = pack_bf16x2(pv[0], pv[1]);
+          pp[w4 * 2 + 1] = pack_bf16x2(pv[2], pv[3]);
+          pd[w4 * 2] = pack_bf16x2(dsv[0], dsv[1]);
+          pd[w4 * 2 + 1] = pack_bf16x2(dsv[2], dsv[3]);
         }
-        // written behind the columns already read: chunk c packs into [16c, 16c+16)
-        tmem_st16(lane_base + C::COL_S + c * 16, pp);
-        tmem_st16(lane_base + C::COL_DP + c * 16, pd);
+        // chunk c packs into [16c, 16c + 16): behind the columns already read
+        tmem_st16(buf + c * 16, pp);
+        tmem_st16(buf + 64 + c * 16, pd);
       }
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(bar(C::BAR_P));
+      if (lane == 0) mbar_arrive(bar(C::BAR_P + wg));
     }
+    // epilogue: warpgroup 0 writes dV, warpgroup 1 writes dK (x scale)
     if (ok && mbar_wait_warp(bar(C::BAR_DONE), 0, ctl)) {
       tc_fence_after();
       const bool store = key < p.N;
       const size_t base = (((size_t)b * p.N + (store ? key : 0)) * p.H_kv + g) * D;
+      __nv_bfloat16* dst = (wg == 0 ? p.dv : p.dk) + base;
+      const float mul = wg == 0 ? 1.0f : p.scale;
+      const uint32_t col0 = wg == 0 ? C::COL_DV : C::COL_DK;
 #pragma unroll
-      for (int which = 0; which < 2; ++which) {
-        __nv_bfloat16* dst = (which == 0 ? p.dv : p.dk) + base;
-        const float mul = which == 0 ? 1.0f : p.scale;
-        const uint32_t col0 = which == 0 ? C::COL_DV : C::COL_DK;
+      for (int c = 0; c < D; c += 32) {
+        uint32_t r[32];
+        tmem_ld32(lane_base + col0 + c, r);
+        uint4 w[4];
+        uint32_t* wp = reinterpret_cast<uint32_t*>(w);
 #pragma unroll
-        for (int c = 0; c < D; c += 32) {
-          uint32_t r[32];
-          tmem_ld32(lane_base + col0 + c, r);  // all lanes: warp-collective
-          uint4 w[4];
-          uint32_t* wp = reinterpret_cast<uint32_t*>(w);
+        for (int x = 0; x < 16; ++x)
+          wp[x] = pack_bf16x2(__uint_as_float(r[2 * x]) * mul, __uint_as_float(r[2 * x + 1]) * mul);
+        if (store) {
+          uint4* d4 = reinterpret_cast<uint4*>(dst + c);
 #pragma unroll
-          for (int x = 0; x < 16; ++x)
-            wp[x] = pack_bf16x2(__uint_as_float(r[2 * x]) * mul, __uint_as_float(r[2 * x + 1]) * mul);
-          if (store) {
-            uint4* d4 = reinterpret_cast<uint4*>(dst + c);
-#pragma unroll
-            for (int x = 0; x < 4; ++x) d4[x] = w[x];
-          }
+          for (int x = 0; x < 4; ++x) d4[x] = w[x];
         }
       }
     }
@@ -309,26 +341,31 @@ __global__ void __launch_bounds__(256, 1)
 template <int D>
 struct DqCfg {
   static constexpr int KCH = D / 64;
-  static constexpr int STAGES = (D == 64) ? 4 : 2;
-  static constexpr int T_BYTES = 128 * D * 2;
-  static constexpr int CHUNK = 128 * 128;
-  static constexpr int STAGE_BYTES = 2 * T_BYTES;     // K_j, V_j
-  static constexpr int OFF_Q = 0, OFF_DO = T_BYTES, OFF_STAGE = 2 * T_BYTES;
+  static constexpr int BK = 64;                        // keys per step
+  static constexpr int STAGES = (D == 64) ? 8 : 4;
+  static constexpr int Q_BYTES = 128 * D * 2;          // Q or dO tile, 128 rows
+  static constexpr int Q_CHUNK = 128 * 128;
+  static constexpr int T_BYTES = BK * D * 2;           // K_j or V_j, 64 keys
+  static constexpr int T_CHUNK = BK * 128;
+  static constexpr int STAGE_BYTES = 2 * T_BYTES;
+  static constexpr int OFF_Q = 0, OFF_DO = Q_BYTES, OFF_STAGE = 2 * Q_BYTES;
   static constexpr int OFF_BAR = OFF_STAGE + STAGES * STAGE_BYTES;
   static constexpr int BAR_QD = 0, BAR_FULL = 1, BAR_EMPTY = 1 + STAGES, BAR_S = 1 + 2 * STAGES,
-                       BAR_P = BAR_S + 1, BAR_DONE = BAR_P + 1, BAR_DRAIN = BAR_DONE + 1, N_BARS = BAR_DRAIN + 1;
+                       BAR_P = BAR_S + 2, BAR_DONE = BAR_P + 2, BAR_DRAIN = BAR_DONE + 1, N_BARS = BAR_DRAIN + 1;
   static constexpr int OFF_MISC = OFF_BAR + N_BARS * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
-  static constexpr int THREADS = 256;
+  static constexpr int THREADS = 384;
   static constexpr uint32_t TMEM_COLS = 512;
-  static constexpr uint32_t COL_S = 0, COL_DP = 128, COL_DQ = 256;
+  static constexpr uint32_t COL_DQ = 256;
+  static_assert(STAGE_BYTES % 1024 == 0, "tile alignment");
 };
 
 // One CTA per 128-row query tile: P heads of one group stacked as in the
 // forward (row r = token_local * P + head offset), so each K/V tile serves all
-// P heads. Warps: 0 TMA, 1 MMA + TMEM owner, 4-7 elementwise (thread = row).
+// P heads. Steps walk 64-key tiles: S = Q K_j^T, dP = dO V_j^T, then
+// dQ += dS K_j with dS read from TMEM.
 template <int D>
-__global__ void __launch_bounds__(256, 1)
+__global__ void __launch_bounds__(384, 1)
     bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
                   const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                   const BwdParams p) {
@@ -359,12 +396,11 @@ __global__ void __launch_bounds__(256, 1)
   const int g = (int)(((long long)head0 * p.H_kv) / p.H_q);
   const int t0 = qt * p.tpt;
   const int t_last = min(p.N - 1, t0 + p.tpt - 1);
-  const int n_kt = (p.N + 127) / 128;
-  const int n_kv = p.causal ? (t_last / 128 + 1) : n_kt;
+  const int n_kv = p.causal ? (t_last / C::BK + 1) : (p.N + C::BK - 1) / C::BK;
 
   WaitCtl ctl{abort_flag, p.status, p.timeout_ns};
   if (tid == 0) {
-    for (int i = 0; i < C::N_BARS; ++i) mbar_init(bar(i), i == C::BAR_P ? 4 : 1);
+    for (int i = 0; i < C::N_BARS; ++i) mbar_init(bar(i), (i == C::BAR_P || i == C::BAR_P + 1) ? 4 : 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -379,22 +415,23 @@ __global__ void __launch_bounds__(256, 1)
 
   if (warp == 0) {
     if (lane == 0) {
-      mbar_arrive_expect_tx(bar(C::BAR_QD), 2 * C::T_BYTES);
+      mbar_arrive_expect_tx(bar(C::BAR_QD), 2 * C::Q_BYTES);
 #pragma unroll
       for (int c = 0; c < C::KCH; ++c) {
-        tma_load_4d(sbase + C::OFF_Q + c * C::CHUNK, &tm_q, bar(C::BAR_QD), c * 64, head0, t0, b);
-        tma_load_4d(sbase + C::OFF_DO + c * C::CHUNK, &tm_do, bar(C::BAR_QD), c * 64, head0, t0, b);
+        tma_load_4d(sbase + C::OFF_Q + c * C::Q_CHUNK, &tm_q, bar(C::BAR_QD), c * 64, head0, t0, b);
+        tma_load_4d(sbase + C::OFF_DO + c * C::Q_CHUNK, &tm_do, bar(C::BAR_QD), c * 64, head0, t0, b);
       }
       int filled = 0;
       for (int j = 0; j < n_kv; ++j) {
         const int st = j % C::STAGES, round = j / C::STAGES;
         if (round > 0 && !mbar_wait(bar(C::BAR_EMPTY + st), (round - 1) & 1, ctl)) break;
         const uint32_t dst = sbase + C::OFF_STAGE + st * C::STAGE_BYTES;
-        mbar_arrive_expect_tx(bar(C::BAR_FULL + st), C::STAGE_BYTES);
+        const uint32_t full = bar(C::BAR_FULL + st);
+        mbar_arrive_expect_tx(full, C::STAGE_BYTES);
 #pragma unroll
         for (int c = 0; c < C::KCH; ++c) {
-          tma_load_4d(dst + c * C::CHUNK, &tm_k, bar(C::BAR_FULL + st), c * 64, g, j * 128, b);
-          tma_load_4d(dst + C::T_BYTES + c * C::CHUNK, &tm_v, bar(C::BAR_FULL + st), c * 64, g, j * 128, b);
+          tma_load_4d(dst + c * C::T_CHUNK, &tm_k, full, c * 64, g, j * C::BK, b);
+          tma_load_4d(dst + C::T_BYTES + c * C::T_CHUNK, &tm_v, full, c * 64, g, j * C::BK, b);
         }
         filled = j + 1;
       }
@@ -406,33 +443,42 @@ __global__ void __launch_bounds__(256, 1)
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      constexpr uint32_t IDESC_S = idesc_bf16_f32(128, 128, 0, 0);
+      constexpr uint32_t IDESC_S = idesc_bf16_f32(128, C::BK, 0, 0);
       constexpr uint32_t IDESC_G = idesc_bf16_f32(128, D, 0, 1);
       const uint32_t qa = sbase + C::OFF_Q, da = sbase + C::OFF_DO;
-      bool ok = mbar_wait(bar(C::BAR_QD), 0, ctl);
-      for (int j = 0; ok && j < n_kv; ++j) {
+      // S = Q K_j^T and dP = dO V_j^T into buffer j & 1
+      auto issue_scores = [&](int j) -> bool {
         const int st = j % C::STAGES;
-        if (!mbar_wait(bar(C::BAR_FULL + st), (j / C::STAGES) & 1, ctl)) { ok = false; break; }
+        if (!mbar_wait(bar(C::BAR_FULL + st), (j / C::STAGES) & 1, ctl)) return false;
         tc_fence_after();
-        const uint32_t ka = sbase + C::OFF_STAGE + st * C::STAGE_BYTES;
-        const uint32_t va = ka + C::T_BYTES;
+        const uint32_t ka = sbase + C::OFF_STAGE + st * C::STAGE_BYTES, va = ka + C::T_BYTES;
+        const uint32_t buf = tmem + (uint32_t)(j & 1) * 128;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * C::CHUNK + (kk & 3) * 32;
-          // S = Q K^T and dP = dO V^T (rows x keys)
-          umma_ss(tmem + C::COL_S, sdesc_sw128(qa + off, 16, 1024), sdesc_sw128(ka + off, 16, 1024), IDESC_S, kk > 0);
-          umma_ss(tmem + C::COL_DP, sdesc_sw128(da + off, 16, 1024), sdesc_sw128(va + off, 16, 1024), IDESC_S,
-                  kk > 0);
+          const uint32_t oq = (kk >> 2) * C::Q_CHUNK + (kk & 3) * 32;
+          const uint32_t ok_ = (kk >> 2) * C::T_CHUNK + (kk & 3) * 32;
+          umma_ss(buf, sdesc_sw128(qa + oq, 16, 1024), sdesc_sw128(ka + ok_, 16, 1024), IDESC_S, kk > 0);
+          umma_ss(buf + 64, sdesc_sw128(da + oq, 16, 1024), sdesc_sw128(va + ok_, 16, 1024), IDESC_S, kk > 0);
         }
-        umma_commit(bar(C::BAR_S));
-        if (!mbar_wait(bar(C::BAR_P), j & 1, ctl)) { ok = false; break; }
+        umma_commit(bar(C::BAR_S + (j & 1)));
+        return true;
+      };
+      bool ok = mbar_wait(bar(C::BAR_QD), 0, ctl);
+      if (ok) ok = issue_scores(0);
+      if (ok && n_kv > 1) ok = issue_scores(1);
+      for (int j = 0; ok && j < n_kv; ++j) {
+        if (!mbar_wait(bar(C::BAR_P + (j & 1)), (j >> 1) & 1, ctl)) { ok = false; break; }
         tc_fence_after();
+        const int st = j % C::STAGES;
+        const uint32_t ka = sbase + C::OFF_STAGE + st * C::STAGE_BYTES;
+        const uint32_t buf = tmem + (uint32_t)(j & 1) * 128;
 #pragma unroll
-        for (int kk = 0; kk < 128 / 16; ++kk)
+        for (int kk = 0; kk < C::BK / 16; ++kk)
           // dQ += dS K_j (K as an MN-major B operand: d contiguous)
-          umma_ts(tmem + C::COL_DQ, tmem + C::COL_S + kk * 8, sdesc_sw128(ka + kk * 16 * 128, C::CHUNK, 1024),
-                  IDESC_G, (j > 0 || kk > 0) ? 1u : 0u);
+          umma_ts(tmem + C::COL_DQ, buf + kk * 8, sdesc_sw128(ka + kk * 16 * 128, C::T_CHUNK, 1024), IDESC_G,
+                  (j > 0 || kk > 0) ? 1u : 0u);
         umma_commit(bar(C::BAR_EMPTY + st));
+        if (j + 2 < n_kv) ok = issue_scores(j + 2);
       }
       if (ok) umma_commit(bar(C::BAR_DONE));
       umma_commit(bar(C::BAR_DRAIN));
@@ -441,12 +487,14 @@ __global__ void __launch_bounds__(256, 1)
       mbar_wait(bar(C::BAR_DRAIN), 0, drain);
     }
   } else if (warp >= 4) {
+    const int wg = (warp - 4) >> 2;
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
     const int token = t0 + (row >> p.log2P);
     const int head = head0 + (row & (p.P - 1));
     const bool row_ok = token < p.N;
     const uint32_t lane_base = tmem + (uint32_t(quarter * 32) << 16);
+    const uint32_t buf = lane_base + (uint32_t)wg * 128;
     const float sl2 = p.scale_log2;
     float lse2_r = 0.f, dsum_r = 0.f;
     if (row_ok) {
@@ -455,15 +503,15 @@ __global__ void __launch_bounds__(256, 1)
       dsum_r = p.dsum[ri];
     }
     bool ok = true;
-    for (int j = 0; j < n_kv; ++j) {
-      if (!mbar_wait_warp(bar(C::BAR_S), j & 1, ctl)) { ok = false; break; }
+    for (int j = wg; j < n_kv; j += 2) {
+      if (!mbar_wait_warp(bar(C::BAR_S + wg), (j >> 1) & 1, ctl)) { ok = false; break; }
       tc_fence_after();
-      const bool need_mask = (j == n_kv - 1) || !row_ok;
+      // keys above t0 only in the last tiles when causal; keys past N in the last tile
+      const bool need_mask = !row_ok || (j * C::BK + C::BK > p.N) || (p.causal && j * C::BK + C::BK - 1 > t0);
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
+      for (int c = 0; c < 2; ++c) {
         uint32_t rs[32], rd[32];
-        tmem_ld32(lane_base + C::COL_S + c * 32, rs);
-        tmem_ld32(lane_base + C::COL_DP + c * 32, rd);
+        tmem_ld32x2(buf + c * 32, buf + 64 + c * 32, rs, rd);
         uint32_t pd[16];
 #pragma unroll
         for (int w = 0; w < 16; ++w) {
@@ -473,25 +521,26 @@ __global__ void __launch_bounds__(256, 1)
             const int col = c * 32 + 2 * w + h;
             float pe = ex2_approx(fmaf(__uint_as_float(rs[2 * w + h]), sl2, -lse2_r));
             if (need_mask) {
-              const int key = j * 128 + col;
+              const int key = j * C::BK + col;
               if (!row_ok || key >= p.N || (p.causal && key > token)) pe = 0.f;
             }
             dv[h] = pe * (__uint_as_float(rd[2 * w + h]) - dsum_r);
           }
           pd[w] = pack_bf16x2(dv[0], dv[1]);
         }
-        tmem_st16(lane_base + C::COL_S + c * 16, pd);
+        tmem_st16(buf + c * 16, pd);
       }
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(bar(C::BAR_P));
+      if (lane == 0) mbar_arrive(bar(C::BAR_P + wg));
     }
+    // epilogue: each warpgroup writes half of the row's d columns (x scale)
     if (ok && mbar_wait_warp(bar(C::BAR_DONE), 0, ctl)) {
       tc_fence_after();
       __nv_bfloat16* dst = p.dq + (((size_t)b * p.N + (row_ok ? token : 0)) * p.H_q + head) * D;
 #pragma unroll
-      for (int c = 0; c < D; c += 32) {
+      for (int c = wg * (D / 2); c < (wg + 1) * (D / 2); c += 32) {
         uint32_t r[32];
         tmem_ld32(lane_base + C::COL_DQ + c, r);
         uint4 w[4];

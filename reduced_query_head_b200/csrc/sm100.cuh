@@ -229,6 +229,27 @@ __device__ __forceinline__ void tmem_ld64(uint32_t taddr, uint32_t (&r)[64]) {
       : "memory");
 }
 
+// Two 32-column loads from different addresses, one wait.
+__device__ __forceinline__ void tmem_ld32x2(uint32_t ta, uint32_t tb, uint32_t (&a)[32], uint32_t (&b)[32]) {
+#define SQA_RA8(x) "=r"(a[x + 0]), "=r"(a[x + 1]), "=r"(a[x + 2]), "=r"(a[x + 3]), \
+                   "=r"(a[x + 4]), "=r"(a[x + 5]), "=r"(a[x + 6]), "=r"(a[x + 7])
+#define SQA_RB8(x) "=r"(b[x + 0]), "=r"(b[x + 1]), "=r"(b[x + 2]), "=r"(b[x + 3]), \
+                   "=r"(b[x + 4]), "=r"(b[x + 5]), "=r"(b[x + 6]), "=r"(b[x + 7])
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%64];\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,"
+      "%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63}, [%65];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : SQA_RA8(0), SQA_RA8(8), SQA_RA8(16), SQA_RA8(24), SQA_RB8(0), SQA_RB8(8), SQA_RB8(16), SQA_RB8(24)
+      : "r"(ta), "r"(tb)
+      : "memory");
+#undef SQA_RA8
+#undef SQA_RB8
+}
+
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "

@@ -141,11 +141,11 @@ int encode_map(CUtensorMap* m, const void* base, int rank, const cuuint64_t* dim
 }
 
 // Tiled fp32 map over `rows` rows of `cols` floats, `ld` floats apart (ld a
-// multiple of 4); boxes of 128 x 1, no swizzle; columns >= cols read as zero.
-int encode_rows_f32(CUtensorMap* m, const float* base, long long rows, int cols, int ld) {
+// multiple of 4); boxes of `box_cols` x 1, no swizzle; columns >= cols read as zero.
+int encode_rows_f32(CUtensorMap* m, const float* base, long long rows, int cols, int ld, int box_cols) {
   const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
   const cuuint64_t strides[1] = {(cuuint64_t)ld * 4};
-  const cuuint32_t box[2] = {128, 1};
+  const cuuint32_t box[2] = {(cuuint32_t)box_cols, 1};
   const cuuint32_t es[2] = {1, 1};
   CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(base), dims, strides, box, es,
                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
@@ -313,11 +313,13 @@ int launch_attn_bwd(const DeviceState* st, const void* q, const void* k, const v
   float* lse2 = reinterpret_cast<float*>(workspace);
   float* dsum = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(workspace) + bwd_vec_bytes(B, N, H_q));
 
-  CUtensorMap tq1, tdo1, tqP, tdoP, tk, tv, tl, td;
+  // dK/dV kernel: Q_j, dO_j of 64 queries of one head, K/V tiles of 128 keys;
+  // dQ kernel: 128-row stacked Q/dO tiles as in the forward, K_j/V_j of 64 keys.
+  CUtensorMap tq1, tdo1, tqP, tdoP, tk128, tv128, tk64, tv64, tl, td;
   {
     const cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)H_q, (cuuint64_t)N, (cuuint64_t)B};
     const cuuint64_t strides[3] = {(cuuint64_t)D * 2, (cuuint64_t)H_q * D * 2, (cuuint64_t)N * H_q * D * 2};
-    const cuuint32_t box1[4] = {64, 1, 128, 1};
+    const cuuint32_t box1[4] = {64, 1, (cuuint32_t)DkdvCfg<D>::BQ, 1};
     const cuuint32_t boxP[4] = {64, (cuuint32_t)P, (cuuint32_t)tpt, 1};
     if (int e = encode_map(&tq1, q, 4, dims, strides, box1)) return e;
     if (int e = encode_map(&tdo1, dout, 4, dims, strides, box1)) return e;
@@ -327,12 +329,15 @@ int launch_attn_bwd(const DeviceState* st, const void* q, const void* k, const v
   {
     const cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)H_kv, (cuuint64_t)N, (cuuint64_t)B};
     const cuuint64_t strides[3] = {(cuuint64_t)D * 2, (cuuint64_t)H_kv * D * 2, (cuuint64_t)N * H_kv * D * 2};
-    const cuuint32_t box[4] = {64, 1, 128, 1};
-    if (int e = encode_map(&tk, k, 4, dims, strides, box)) return e;
-    if (int e = encode_map(&tv, v, 4, dims, strides, box)) return e;
+    const cuuint32_t box128[4] = {64, 1, 128, 1};
+    const cuuint32_t box64[4] = {64, 1, (cuuint32_t)DqCfg<D>::BK, 1};
+    if (int e = encode_map(&tk128, k, 4, dims, strides, box128)) return e;
+    if (int e = encode_map(&tv128, v, 4, dims, strides, box128)) return e;
+    if (int e = encode_map(&tk64, k, 4, dims, strides, box64)) return e;
+    if (int e = encode_map(&tv64, v, 4, dims, strides, box64)) return e;
   }
-  if (int e = encode_rows_f32(&tl, lse2, (long long)B * H_q, N, ld)) return e;
-  if (int e = encode_rows_f32(&td, dsum, (long long)B * H_q, N, ld)) return e;
+  if (int e = encode_rows_f32(&tl, lse2, (long long)B * H_q, N, ld, DkdvCfg<D>::BQ)) return e;
+  if (int e = encode_rows_f32(&td, dsum, (long long)B * H_q, N, ld, DkdvCfg<D>::BQ)) return e;
 
   BwdParams p;
   p.dq = reinterpret_cast<__nv_bfloat16*>(dq);
@@ -360,9 +365,9 @@ int launch_attn_bwd(const DeviceState* st, const void* q, const void* k, const v
       N, H_q, ld);
   if (cudaGetLastError() != cudaSuccess) return SQA_ERR_CUDA;
   sqa::bwd_dkdv_kernel<D><<<(unsigned)grid_kv, DkdvCfg<D>::THREADS, DkdvCfg<D>::SMEM_BYTES, stream>>>(
-      tq1, tdo1, tk, tv, tl, td, p);
+      tq1, tdo1, tk128, tv128, tl, td, p);
   if (cudaGetLastError() != cudaSuccess) return SQA_ERR_CUDA;
-  sqa::bwd_dq_kernel<D><<<(unsigned)grid_q, DqCfg<D>::THREADS, DqCfg<D>::SMEM_BYTES, stream>>>(tqP, tdoP, tk, tv, p);
+  sqa::bwd_dq_kernel<D><<<(unsigned)grid_q, DqCfg<D>::THREADS, DqCfg<D>::SMEM_BYTES, stream>>>(tqP, tdoP, tk64, tv64, p);
   return cudaGetLastError() == cudaSuccess ? SQA_OK : SQA_ERR_CUDA;
 }
 
