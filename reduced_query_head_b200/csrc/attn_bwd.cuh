@@ -202,20 +202,26 @@ __global__ void __launch_bounds__(384, 1)
     if (lane == 0) {
       constexpr uint32_t IDESC_S = idesc_bf16_f32(128, C::BQ, 0, 0);
       constexpr uint32_t IDESC_G = idesc_bf16_f32(128, D, 0, 1);
-      const uint32_t ka = sbase + C::OFF_K, va = sbase + C::OFF_V;
+      // Descriptors are built once; a byte offset `o` inside shared memory is
+      // added as o >> 4 to the start-address field (no carry: smem < 256 KB).
+      const uint64_t dK = sdesc_sw128(sbase + C::OFF_K, 16, 1024), dV = sdesc_sw128(sbase + C::OFF_V, 16, 1024);
+      const uint64_t dQk = sdesc_sw128(sbase + C::OFF_STAGE, 16, 1024);
+      const uint64_t dDk = sdesc_sw128(sbase + C::OFF_STAGE + C::T_BYTES, 16, 1024);
+      const uint64_t dQm = sdesc_sw128(sbase + C::OFF_STAGE, C::T_CHUNK, 1024);
+      const uint64_t dDm = sdesc_sw128(sbase + C::OFF_STAGE + C::T_BYTES, C::T_CHUNK, 1024);
       // S^T = K Q_s^T and dP^T = V dO_s^T into buffer s & 1
       auto issue_scores = [&](int s) -> bool {
         const int st = s % C::STAGES;
         if (!mbar_wait(bar(C::BAR_FULL + st), (s / C::STAGES) & 1, ctl)) return false;
         tc_fence_after();
-        const uint32_t qa = sbase + C::OFF_STAGE + st * C::STAGE_BYTES, da = qa + C::T_BYTES;
+        const uint64_t so = (uint64_t)(st * (C::STAGE_BYTES >> 4));
         const uint32_t buf = tmem + (uint32_t)(s & 1) * 128;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t ok_ = (kk >> 2) * C::KV_CHUNK + (kk & 3) * 32;
-          const uint32_t oq = (kk >> 2) * C::T_CHUNK + (kk & 3) * 32;
-          umma_ss(buf, sdesc_sw128(ka + ok_, 16, 1024), sdesc_sw128(qa + oq, 16, 1024), IDESC_S, kk > 0);
-          umma_ss(buf + 64, sdesc_sw128(va + ok_, 16, 1024), sdesc_sw128(da + oq, 16, 1024), IDESC_S, kk > 0);
+          const uint64_t ok_ = ((kk >> 2) * C::KV_CHUNK + (kk & 3) * 32) >> 4;
+          const uint64_t oq = ((kk >> 2) * C::T_CHUNK + (kk & 3) * 32) >> 4;
+          umma_ss(buf, dK + ok_, dQk + so + oq, IDESC_S, kk > 0);
+          umma_ss(buf + 64, dV + ok_, dDk + so + oq, IDESC_S, kk > 0);
         }
         umma_commit(bar(C::BAR_S + (s & 1)));
         return true;
@@ -227,15 +233,15 @@ __global__ void __launch_bounds__(384, 1)
         if (!mbar_wait(bar(C::BAR_P + (s & 1)), (s >> 1) & 1, ctl)) { ok = false; break; }
         tc_fence_after();
         const int st = s % C::STAGES;
-        const uint32_t qa = sbase + C::OFF_STAGE + st * C::STAGE_BYTES, da = qa + C::T_BYTES;
+        const uint64_t so = (uint64_t)(st * (C::STAGE_BYTES >> 4));
         const uint32_t buf = tmem + (uint32_t)(s & 1) * 128;
 #pragma unroll
         for (int kk = 0; kk < C::BQ / 16; ++kk) {
           const uint32_t acc = (s > 0 || kk > 0) ? 1u : 0u;
+          const uint64_t ob = (uint64_t)((kk * 16 * 128) >> 4);
           // dV += P^T dO_s and dK += dS^T Q_s (B operands MN-major: d contiguous)
-          umma_ts(tmem + C::COL_DV, buf + kk * 8, sdesc_sw128(da + kk * 16 * 128, C::T_CHUNK, 1024), IDESC_G, acc);
-          umma_ts(tmem + C::COL_DK, buf + 64 + kk * 8, sdesc_sw128(qa + kk * 16 * 128, C::T_CHUNK, 1024), IDESC_G,
-                  acc);
+          umma_ts(tmem + C::COL_DV, buf + kk * 8, dDm + so + ob, IDESC_G, acc);
+          umma_ts(tmem + C::COL_DK, buf + 64 + kk * 8, dQm + so + ob, IDESC_G, acc);
         }
         umma_commit(bar(C::BAR_EMPTY + st));
         if (s + 2 < n_steps) ok = issue_scores(s + 2);
@@ -272,6 +278,15 @@ __global__ void __launch_bounds__(384, 1)
       for (int c = 0; c < 2; ++c) {
         uint32_t rs[32], rd[32];
         tmem_ld32x2(buf + c * 32, buf + 64 + c * 32, rs, rd);
+        // masked scores become -inf (p = 0) in a pass of their own, so the
+        // arithmetic below stays one straight block
+        if (need_mask) {
+#pragma unroll
+          for (int x = 0; x < 32; ++x) {
+            const int q = t * C::BQ + c * 32 + x;
+            if (q >= p.N || key >= p.N || (p.causal && key > q)) rs[x] = __float_as_uint(-INFINITY);
+          }
+        }
         uint32_t pp[16], pd[16];
 #pragma unroll
         for (int w4 = 0; w4 < 8; ++w4) {
@@ -280,12 +295,7 @@ __global__ void __launch_bounds__(384, 1)
           float pv[4], dsv[4];
 #pragma unroll
           for (int h = 0; h < 4; ++h) {
-            const int col = c * 32 + w4 * 4 + h;
-            float pe = ex2_approx(fmaf(__uint_as_float(rs[w4 * 4 + h]), sl2, -lv[h]));
-            if (need_mask) {
-              const int q = t * C::BQ + col;
-              if (q >= p.N || key >= p.N || (p.causal && key > q)) pe = 0.f;
-            }
+            const float pe = ex2_approx(fmaf(__uint_as_float(rs[w4 * 4 + h]), sl2, -lv[h]));
             pv[h] = pe;
             dsv[h] = pe * (__uint_as_float(rd[w4 * 4 + h]) - dv_[h]);
           }
@@ -445,20 +455,24 @@ __global__ void __launch_bounds__(384, 1)
     if (lane == 0) {
       constexpr uint32_t IDESC_S = idesc_bf16_f32(128, C::BK, 0, 0);
       constexpr uint32_t IDESC_G = idesc_bf16_f32(128, D, 0, 1);
-      const uint32_t qa = sbase + C::OFF_Q, da = sbase + C::OFF_DO;
+      // descriptors built once; offsets added as o >> 4 (see the dK/dV kernel)
+      const uint64_t dQ = sdesc_sw128(sbase + C::OFF_Q, 16, 1024), dO = sdesc_sw128(sbase + C::OFF_DO, 16, 1024);
+      const uint64_t dKk = sdesc_sw128(sbase + C::OFF_STAGE, 16, 1024);
+      const uint64_t dVk = sdesc_sw128(sbase + C::OFF_STAGE + C::T_BYTES, 16, 1024);
+      const uint64_t dKm = sdesc_sw128(sbase + C::OFF_STAGE, C::T_CHUNK, 1024);
       // S = Q K_j^T and dP = dO V_j^T into buffer j & 1
       auto issue_scores = [&](int j) -> bool {
         const int st = j % C::STAGES;
         if (!mbar_wait(bar(C::BAR_FULL + st), (j / C::STAGES) & 1, ctl)) return false;
         tc_fence_after();
-        const uint32_t ka = sbase + C::OFF_STAGE + st * C::STAGE_BYTES, va = ka + C::T_BYTES;
+        const uint64_t so = (uint64_t)(st * (C::STAGE_BYTES >> 4));
         const uint32_t buf = tmem + (uint32_t)(j & 1) * 128;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t oq = (kk >> 2) * C::Q_CHUNK + (kk & 3) * 32;
-          const uint32_t ok_ = (kk >> 2) * C::T_CHUNK + (kk & 3) * 32;
-          umma_ss(buf, sdesc_sw128(qa + oq, 16, 1024), sdesc_sw128(ka + ok_, 16, 1024), IDESC_S, kk > 0);
-          umma_ss(buf + 64, sdesc_sw128(da + oq, 16, 1024), sdesc_sw128(va + ok_, 16, 1024), IDESC_S, kk > 0);
+          const uint64_t oq = ((kk >> 2) * C::Q_CHUNK + (kk & 3) * 32) >> 4;
+          const uint64_t ok_ = ((kk >> 2) * C::T_CHUNK + (kk & 3) * 32) >> 4;
+          umma_ss(buf, dQ + oq, dKk + so + ok_, IDESC_S, kk > 0);
+          umma_ss(buf + 64, dO + oq, dVk + so + ok_, IDESC_S, kk > 0);
         }
         umma_commit(bar(C::BAR_S + (j & 1)));
         return true;
@@ -470,12 +484,12 @@ __global__ void __launch_bounds__(384, 1)
         if (!mbar_wait(bar(C::BAR_P + (j & 1)), (j >> 1) & 1, ctl)) { ok = false; break; }
         tc_fence_after();
         const int st = j % C::STAGES;
-        const uint32_t ka = sbase + C::OFF_STAGE + st * C::STAGE_BYTES;
+        const uint64_t so = (uint64_t)(st * (C::STAGE_BYTES >> 4));
         const uint32_t buf = tmem + (uint32_t)(j & 1) * 128;
 #pragma unroll
         for (int kk = 0; kk < C::BK / 16; ++kk)
           // dQ += dS K_j (K as an MN-major B operand: d contiguous)
-          umma_ts(tmem + C::COL_DQ, buf + kk * 8, sdesc_sw128(ka + kk * 16 * 128, C::T_CHUNK, 1024), IDESC_G,
+          umma_ts(tmem + C::COL_DQ, buf + kk * 8, dKm + so + (uint64_t)((kk * 16 * 128) >> 4), IDESC_G,
                   (j > 0 || kk > 0) ? 1u : 0u);
         umma_commit(bar(C::BAR_EMPTY + st));
         if (j + 2 < n_kv) ok = issue_scores(j + 2);
@@ -512,18 +526,20 @@ __global__ void __launch_bounds__(384, 1)
       for (int c = 0; c < 2; ++c) {
         uint32_t rs[32], rd[32];
         tmem_ld32x2(buf + c * 32, buf + 64 + c * 32, rs, rd);
+        if (need_mask) {   // masked scores -> -inf (p = 0), outside the arithmetic block
+#pragma unroll
+          for (int x = 0; x < 32; ++x) {
+            const int key = j * C::BK + c * 32 + x;
+            if (!row_ok || key >= p.N || (p.causal && key > token)) rs[x] = __float_as_uint(-INFINITY);
+          }
+        }
         uint32_t pd[16];
 #pragma unroll
         for (int w = 0; w < 16; ++w) {
           float dv[2];
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
-            const int col = c * 32 + 2 * w + h;
-            float pe = ex2_approx(fmaf(__uint_as_float(rs[2 * w + h]), sl2, -lse2_r));
-            if (need_mask) {
-              const int key = j * C::BK + col;
-              if (!row_ok || key >= p.N || (p.causal && key > token)) pe = 0.f;
-            }
+            const float pe = ex2_approx(fmaf(__uint_as_float(rs[2 * w + h]), sl2, -lse2_r));
             dv[h] = pe * (__uint_as_float(rd[2 * w + h]) - dsum_r);
           }
           pd[w] = pack_bf16x2(dv[0], dv[1]);
