@@ -24,14 +24,16 @@
 namespace sqa {
 
 // ---------------------------------------------------------------- prep
-// One warp per row (b, t, i): D = sum_c dO * O (fp32), lse2 = lse * log2(e).
-// Both outputs are [B * H_q] rows of `ld` >= N floats (ld a multiple of 4, so
-// that the rows can be TMA-loaded); columns >= N are never written.
+// One warp per row (b, t, i): D = sum_c dO * O (fp32) and lse2 = lse * log2(e),
+// both stored negated (-D, -lse2) so that the main kernels add them with a
+// plain fused multiply-add. Outputs are [B * H_q] rows of `ld` >= N floats (ld
+// a multiple of 4, so that the rows can be TMA-loaded); columns >= N are never
+// written.
 template <int D>
 __global__ void __launch_bounds__(256) bwd_prep_kernel(const __nv_bfloat16* __restrict__ out,
                                                        const __nv_bfloat16* __restrict__ dout,
-                                                       const float* __restrict__ lse, float* __restrict__ dsum,
-                                                       float* __restrict__ lse2, int B, int N, int H_q, int ld) {
+                                                       const float* __restrict__ lse, float* __restrict__ ndsum,
+                                                       float* __restrict__ nlse2, int B, int N, int H_q, int ld) {
   const long long rows = (long long)B * N * H_q;
   const long long row = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
@@ -49,17 +51,21 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const __nv_bfloat16* __re
     const long long i = row % H_q;
     const long long bt = row / H_q;
     const long long t = bt % N, b = bt / N;
-    dsum[(b * H_q + i) * ld + t] = acc;
-    lse2[(b * H_q + i) * ld + t] = lse[(b * H_q + i) * N + t] * 1.4426950408889634f;
+    ndsum[(b * H_q + i) * ld + t] = -acc;
+    nlse2[(b * H_q + i) * ld + t] = lse[(b * H_q + i) * N + t] * -1.4426950408889634f;
   }
 }
 
 struct BwdParams {
+  const __nv_bfloat16* q;     // [B, N, H_q, D]
+  const __nv_bfloat16* k;     // [B, N, H_kv, D]
+  const __nv_bfloat16* v;     // [B, N, H_kv, D]
+  const __nv_bfloat16* dout;  // [B, N, H_q, D]
   __nv_bfloat16* dq;    // [B, N, H_q, D]
   __nv_bfloat16* dk;    // [B, N, H_kv, D]
   __nv_bfloat16* dv;    // [B, N, H_kv, D]
-  const float* lse2;    // [B, H_q] rows of ld: log-sum-exp in log2 units
-  const float* dsum;    // [B, H_q] rows of ld: rowsum(dO * O)
+  const float* nlse2;   // [B, H_q] rows of ld: -(log-sum-exp in log2 units)
+  const float* ndsum;   // [B, H_q] rows of ld: -rowsum(dO * O)
   int ld;               // row stride of lse2 / dsum
   int B, N, H_q, H_kv;
   int P, log2P, tpt;    // dq kernel: heads stacked per tile, tokens per tile
@@ -72,40 +78,65 @@ struct BwdParams {
 };
 
 
+
 // Both main kernels run a two-buffer pipeline over 64-column steps. TMEM
 // buffer b (b = step & 1) holds the step's scores in [128b, 128b + 64) and
 // its dP in [128b + 64, 128b + 128); the elementwise warpgroup that owns the
 // buffer writes P / dS back as bf16 over the first 32 columns of each half.
-// The MMA thread issues step s + 2's score products right after step s's
-// gradient products, so the tensor core works on one buffer while a
-// warpgroup works on the other.
+// Each buffer has its own MMA issuer (warp 1 for even steps, warp 3 for odd
+// steps) with its own gradient accumulators, summed in the epilogue: while one
+// issuer waits for its warpgroup, the other's products keep the tensor core
+// busy. (The dK/dV kernel at d = 128 has no TMEM left for a second set of
+// accumulators and runs one issuer over both buffers.)
 //   warp 0      TMA producer
-//   warp 1      MMA issuer + TMEM owner
+//   warp 1      MMA issuer 0 + TMEM owner
+//   warp 3      MMA issuer 1
 //   warps 4-7   elementwise for even steps (thread = TMEM lane = tile row)
 //   warps 8-11  elementwise for odd steps
+
+// 16 columns of the elementwise step from the scores s and dP read from TMEM:
+// p = exp2(s * scale_log2 - lse2), ds = p * (dP - D), both packed to bf16
+// pairs (low half = even column). nl / nd hold -lse2 / -D per column pair.
+__device__ __forceinline__ void bwd_chunk(const uint32_t (&rs)[16], const uint32_t (&rd)[16], float sl2,
+                                          const float2 (&nl)[8], const float2 (&nd)[8], uint32_t (&pp)[8],
+                                          uint32_t (&pd)[8]) {
+  const float2 s2 = make_float2(sl2, sl2);
+#pragma unroll
+  for (int w = 0; w < 8; ++w) {
+    const float2 x = ffma2(make_float2(__uint_as_float(rs[2 * w]), __uint_as_float(rs[2 * w + 1])), s2, nl[w]);
+    const float2 pe = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+    const float2 g = fadd2(make_float2(__uint_as_float(rd[2 * w]), __uint_as_float(rd[2 * w + 1])), nd[w]);
+    const float2 ds = fmul2(pe, g);
+    pp[w] = pack_bf16x2(pe.x, pe.y);
+    pd[w] = pack_bf16x2(ds.x, ds.y);
+  }
+}
 
 // ---------------------------------------------------------------- dK, dV
 template <int D>
 struct DkdvCfg {
   static constexpr int KCH = D / 64;                   // 128-byte column chunks
   static constexpr int BQ = 64;                        // queries per step
+  static constexpr int NI = (D == 64) ? 2 : 1;         // MMA issuers (see above)
   static constexpr int STAGES = (D == 64) ? 8 : 4;
   static constexpr int KV_BYTES = 128 * D * 2;         // K or V tile, 128 keys
   static constexpr int KV_CHUNK = 128 * 128;           // one column chunk of it
   static constexpr int T_BYTES = BQ * D * 2;           // Q_j or dO_j, 64 queries
   static constexpr int T_CHUNK = BQ * 128;
   static constexpr int STAGE_BYTES = 2 * T_BYTES;
-  static constexpr int VEC_BYTES = BQ * 4;             // lse2 or dsum of the step's queries
+  static constexpr int VEC_BYTES = BQ * 4;             // -lse2 or -D of the step's queries
   static constexpr int OFF_K = 0, OFF_V = KV_BYTES, OFF_STAGE = 2 * KV_BYTES;
-  static constexpr int OFF_VEC = OFF_STAGE + STAGES * STAGE_BYTES;   // [STAGES][lse2 | dsum]
+  static constexpr int OFF_VEC = OFF_STAGE + STAGES * STAGE_BYTES;   // [STAGES][-lse2 | -D]
   static constexpr int OFF_BAR = OFF_VEC + STAGES * 2 * VEC_BYTES;
   static constexpr int BAR_KV = 0, BAR_FULL = 1, BAR_EMPTY = 1 + STAGES, BAR_S = 1 + 2 * STAGES,
-                       BAR_P = BAR_S + 2, BAR_DONE = BAR_P + 2, BAR_DRAIN = BAR_DONE + 1, N_BARS = BAR_DRAIN + 1;
+                       BAR_P = BAR_S + 2, BAR_DONE = BAR_P + 2, BAR_DRAIN = BAR_DONE + 2, N_BARS = BAR_DRAIN + 2;
   static constexpr int OFF_MISC = OFF_BAR + N_BARS * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
   static constexpr int THREADS = 384;
   static constexpr uint32_t TMEM_COLS = 512;
-  static constexpr uint32_t COL_DV = 256, COL_DK = 256 + D;
+  // accumulators of issuer i: dV at COL_ACC + i * ACC_STRIDE, dK D columns after it
+  static constexpr uint32_t COL_ACC = 256, ACC_STRIDE = 2 * D;
+  static_assert(COL_ACC + NI * ACC_STRIDE <= TMEM_COLS, "TMEM budget");
   static_assert(STAGE_BYTES % 1024 == 0 && OFF_STAGE % 1024 == 0, "tile alignment");
 };
 
@@ -198,8 +229,9 @@ __global__ void __launch_bounds__(384, 1)
       for (int s = max(0, filled - C::STAGES); s < filled; ++s)
         mbar_wait(bar(C::BAR_FULL + s % C::STAGES), (s / C::STAGES) & 1, drain);
     }
-  } else if (warp == 1) {
+  } else if (warp == 1 || (C::NI == 2 && warp == 3)) {
     if (lane == 0) {
+      const int me = warp == 1 ? 0 : 1;
       constexpr uint32_t IDESC_S = idesc_bf16_f32(128, C::BQ, 0, 0);
       constexpr uint32_t IDESC_G = idesc_bf16_f32(128, D, 0, 1);
       // Descriptors are built once; a byte offset `o` inside shared memory is
@@ -227,30 +259,35 @@ __global__ void __launch_bounds__(384, 1)
         return true;
       };
       bool ok = mbar_wait(bar(C::BAR_KV), 0, ctl);
-      if (ok) ok = issue_scores(0);
-      if (ok && n_steps > 1) ok = issue_scores(1);
-      for (int s = 0; ok && s < n_steps; ++s) {
-        if (!mbar_wait(bar(C::BAR_P + (s & 1)), (s >> 1) & 1, ctl)) { ok = false; break; }
+      if (C::NI == 2) {
+        if (ok && me < n_steps) ok = issue_scores(me);
+      } else {
+        if (ok) ok = issue_scores(0);
+        if (ok && n_steps > 1) ok = issue_scores(1);
+      }
+      const uint32_t col_dv = tmem + C::COL_ACC + (uint32_t)me * C::ACC_STRIDE, col_dk = col_dv + D;
+      for (int s = me; ok && s < n_steps; s += C::NI) {
+        if (!mbar_wait_spin(bar(C::BAR_P + (s & 1)), (s >> 1) & 1, ctl)) { ok = false; break; }
         tc_fence_after();
         const int st = s % C::STAGES;
         const uint64_t so = (uint64_t)(st * (C::STAGE_BYTES >> 4));
         const uint32_t buf = tmem + (uint32_t)(s & 1) * 128;
 #pragma unroll
         for (int kk = 0; kk < C::BQ / 16; ++kk) {
-          const uint32_t acc = (s > 0 || kk > 0) ? 1u : 0u;
+          const uint32_t acc = (s > me || kk > 0) ? 1u : 0u;
           const uint64_t ob = (uint64_t)((kk * 16 * 128) >> 4);
           // dV += P^T dO_s and dK += dS^T Q_s (B operands MN-major: d contiguous)
-          umma_ts(tmem + C::COL_DV, buf + kk * 8, dDm + so + ob, IDESC_G, acc);
-          umma_ts(tmem + C::COL_DK, buf + 64 + kk * 8, dQm + so + ob, IDESC_G, acc);
+          umma_ts(col_dv, buf + kk * 8, dDm + so + ob, IDESC_G, acc);
+          umma_ts(col_dk, buf + 64 + kk * 8, dQm + so + ob, IDESC_G, acc);
         }
         umma_commit(bar(C::BAR_EMPTY + st));
         if (s + 2 < n_steps) ok = issue_scores(s + 2);
       }
-      if (ok) umma_commit(bar(C::BAR_DONE));
-      umma_commit(bar(C::BAR_DRAIN));
+      if (ok) umma_commit(bar(C::BAR_DONE + me));
+      umma_commit(bar(C::BAR_DRAIN + me));
       volatile int zero = 0;
       WaitCtl drain{&zero, p.status, drain_limit_ns(p.timeout_ns)};
-      mbar_wait(bar(C::BAR_DRAIN), 0, drain);
+      mbar_wait(bar(C::BAR_DRAIN + me), 0, drain);
     }
   } else if (warp >= 4) {
     const int wg = (warp - 4) >> 2;          // 0: even steps, 1: odd steps
@@ -264,8 +301,12 @@ __global__ void __launch_bounds__(384, 1)
     for (int s = wg; s < n_steps; s += 2) {
       const int st = s % C::STAGES;
       const int t = t_start + s % per_head;
+      // The two warpgroups take turns: step s starts once step s - 1 is done,
+      // so each runs alone while the tensor core works on the other buffer
+      // (run together, they finish together and leave the tensor core idle).
       if (!mbar_wait_warp(bar(C::BAR_S + wg), (s >> 1) & 1, ctl) ||
-          !mbar_wait_warp(bar(C::BAR_FULL + st), (s / C::STAGES) & 1, ctl)) {
+          !mbar_wait_warp(bar(C::BAR_FULL + st), (s / C::STAGES) & 1, ctl) ||
+          (s > 0 && !mbar_wait_warp(bar(C::BAR_P + (wg ^ 1)), ((s - 1) >> 1) & 1, ctl))) {
         ok = false;
         break;
       }
@@ -274,57 +315,68 @@ __global__ void __launch_bounds__(384, 1)
       const float4* vd4 = vl4 + C::BQ / 4;
       // a key above a query of the step only on the two diagonal tiles; ragged ends
       const bool need_mask = (p.causal && t < 2 * u + 2) || (t * C::BQ + C::BQ > p.N) || (key >= p.N);
+      // four 16-column chunks; chunk k + 1's TMEM load is in flight while
+      // chunk k is computed
+      uint32_t a0[16], b0[16], a1[16], b1[16];
+      tmem_ld16x2_nowait(buf, buf + 64, a0, b0);
+      tmem_ld_wait16x2(a0, b0);
 #pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        uint32_t rs[32], rd[32];
-        tmem_ld32x2(buf + c * 32, buf + 64 + c * 32, rs, rd);
+      for (int k = 0; k < 4; ++k) {
+        uint32_t(&ra)[16] = (k & 1) ? a1 : a0;
+        uint32_t(&rb)[16] = (k & 1) ? b1 : b0;
+        uint32_t(&na)[16] = (k & 1) ? a0 : a1;
+        uint32_t(&nb)[16] = (k & 1) ? b0 : b1;
+        if (k < 3) tmem_ld16x2_nowait(buf + 16 * (k + 1), buf + 64 + 16 * (k + 1), na, nb);
         // masked scores become -inf (p = 0) in a pass of their own, so the
-        // arithmetic below stays one straight block
+        // arithmetic stays one straight block
         if (need_mask) {
 #pragma unroll
-          for (int x = 0; x < 32; ++x) {
-            const int q = t * C::BQ + c * 32 + x;
-            if (q >= p.N || key >= p.N || (p.causal && key > q)) rs[x] = __float_as_uint(-INFINITY);
+          for (int x = 0; x < 16; ++x) {
+            const int q = t * C::BQ + k * 16 + x;
+            if (q >= p.N || key >= p.N || (p.causal && key > q)) ra[x] = __float_as_uint(-INFINITY);
           }
         }
-        uint32_t pp[16], pd[16];
+        float2 nl[8], nd[8];
 #pragma unroll
-        for (int w4 = 0; w4 < 8; ++w4) {
-          const float4 l4 = vl4[c * 8 + w4], d4 = vd4[c * 8 + w4];
-          const float lv[4] = {l4.x, l4.y, l4.z, l4.w}, dv_[4] = {d4.x, d4.y, d4.z, d4.w};
-          float pv[4], dsv[4];
-#pragma unroll
-          for (int h = 0; h < 4; ++h) {
-            const float pe = ex2_approx(fmaf(__uint_as_float(rs[w4 * 4 + h]), sl2, -lv[h]));
-            pv[h] = pe;
-            dsv[h] = pe * (__uint_as_float(rd[w4 * 4 + h]) - dv_[h]);
-          }
-          pp[w4 * 2] = pack_bf16x2(pv[0], pv[1]);
-          pp[w4 * 2 + 1] = pack_bf16x2(pv[2], pv[3]);
-          pd[w4 * 2] = pack_bf16x2(dsv[0], dsv[1]);
-          pd[w4 * 2 + 1] = pack_bf16x2(dsv[2], dsv[3]);
+        for (int w = 0; w < 4; ++w) {
+          const float4 l4 = vl4[k * 4 + w], d4 = vd4[k * 4 + w];
+          nl[2 * w] = make_float2(l4.x, l4.y);
+          nl[2 * w + 1] = make_float2(l4.z, l4.w);
+          nd[2 * w] = make_float2(d4.x, d4.y);
+          nd[2 * w + 1] = make_float2(d4.z, d4.w);
         }
-        // chunk c packs into [16c, 16c + 16): behind the columns already read
-        tmem_st16(buf + c * 16, pp);
-        tmem_st16(buf + 64 + c * 16, pd);
+        uint32_t pp[8], pd[8];
+        bwd_chunk(ra, rb, sl2, nl, nd, pp, pd);
+        // chunk k packs into [8k, 8k + 8): behind the columns already read
+        tmem_st8(buf + k * 8, pp);
+        tmem_st8(buf + 64 + k * 8, pd);
+        if (k < 3) tmem_ld_wait16x2(na, nb);
       }
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(C::BAR_P + wg));
     }
-    // epilogue: warpgroup 0 writes dV, warpgroup 1 writes dK (x scale)
-    if (ok && mbar_wait_warp(bar(C::BAR_DONE), 0, ctl)) {
+    // epilogue: warpgroup 0 writes dV, warpgroup 1 writes dK (x scale), each
+    // the sum over the issuers' accumulators
+    const bool two = C::NI == 2 && n_steps > 1;
+    if (ok && mbar_wait_warp(bar(C::BAR_DONE), 0, ctl) && (!two || mbar_wait_warp(bar(C::BAR_DONE + 1), 0, ctl))) {
       tc_fence_after();
       const bool store = key < p.N;
       const size_t base = (((size_t)b * p.N + (store ? key : 0)) * p.H_kv + g) * D;
       __nv_bfloat16* dst = (wg == 0 ? p.dv : p.dk) + base;
       const float mul = wg == 0 ? 1.0f : p.scale;
-      const uint32_t col0 = wg == 0 ? C::COL_DV : C::COL_DK;
+      const uint32_t col0 = lane_base + C::COL_ACC + (wg == 0 ? 0u : (uint32_t)D);
 #pragma unroll
       for (int c = 0; c < D; c += 32) {
-        uint32_t r[32];
-        tmem_ld32(lane_base + col0 + c, r);
+        uint32_t r[32], r1[32];
+        if (two) {
+          tmem_ld32x2(col0 + c, col0 + C::ACC_STRIDE + c, r, r1);
+#pragma unroll
+          for (int x = 0; x < 32; ++x) r[x] = __float_as_uint(__uint_as_float(r[x]) + __uint_as_float(r1[x]));
+        } else {
+          tmem_ld32(col0 + c, r);
+        }
         uint4 w[4];
         uint32_t* wp = reinterpret_cast<uint32_t*>(w);
 #pragma unroll
@@ -353,21 +405,27 @@ struct DqCfg {
   static constexpr int KCH = D / 64;
   static constexpr int BK = 64;                        // keys per step
   static constexpr int STAGES = (D == 64) ? 8 : 4;
+  // d = 64: Q and dO live in TMEM as the A operands of the score products (TS
+  // form); at d = 128 the two issuers' accumulators fill TMEM and they stay in
+  // shared memory.
+  static constexpr bool A_TMEM = (D == 64);
   static constexpr int Q_BYTES = 128 * D * 2;          // Q or dO tile, 128 rows
   static constexpr int Q_CHUNK = 128 * 128;
   static constexpr int T_BYTES = BK * D * 2;           // K_j or V_j, 64 keys
   static constexpr int T_CHUNK = BK * 128;
   static constexpr int STAGE_BYTES = 2 * T_BYTES;
-  static constexpr int OFF_Q = 0, OFF_DO = Q_BYTES, OFF_STAGE = 2 * Q_BYTES;
+  static constexpr int OFF_Q = 0, OFF_DO = Q_BYTES, OFF_STAGE = A_TMEM ? 0 : 2 * Q_BYTES;
   static constexpr int OFF_BAR = OFF_STAGE + STAGES * STAGE_BYTES;
   static constexpr int BAR_QD = 0, BAR_FULL = 1, BAR_EMPTY = 1 + STAGES, BAR_S = 1 + 2 * STAGES,
-                       BAR_P = BAR_S + 2, BAR_DONE = BAR_P + 2, BAR_DRAIN = BAR_DONE + 1, N_BARS = BAR_DRAIN + 1;
+                       BAR_P = BAR_S + 2, BAR_DONE = BAR_P + 2, BAR_DRAIN = BAR_DONE + 2, N_BARS = BAR_DRAIN + 2;
   static constexpr int OFF_MISC = OFF_BAR + N_BARS * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
   static constexpr int THREADS = 384;
   static constexpr uint32_t TMEM_COLS = 512;
-  static constexpr uint32_t COL_DQ = 256;
-  static_assert(STAGE_BYTES % 1024 == 0, "tile alignment");
+  // dQ accumulator of issuer i at COL_DQ + i * D; Q / dO rows (A_TMEM) after them
+  static constexpr uint32_t COL_DQ = 256, COL_QT = 256 + 2 * D, COL_DOT = COL_QT + D / 2;
+  static_assert(COL_DQ + 2 * D <= TMEM_COLS && (!A_TMEM || COL_DOT + D / 2 <= TMEM_COLS), "TMEM budget");
+  static_assert(STAGE_BYTES % 1024 == 0 && OFF_STAGE % 1024 == 0, "tile alignment");
 };
 
 // One CTA per 128-row query tile: P heads of one group stacked as in the
@@ -410,7 +468,8 @@ __global__ void __launch_bounds__(384, 1)
 
   WaitCtl ctl{abort_flag, p.status, p.timeout_ns};
   if (tid == 0) {
-    for (int i = 0; i < C::N_BARS; ++i) mbar_init(bar(i), (i == C::BAR_P || i == C::BAR_P + 1) ? 4 : 1);
+    for (int i = 0; i < C::N_BARS; ++i)
+      mbar_init(bar(i), (i == C::BAR_P || i == C::BAR_P + 1) ? 4 : ((C::A_TMEM && i == C::BAR_QD) ? 8 : 1));
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -425,11 +484,13 @@ __global__ void __launch_bounds__(384, 1)
 
   if (warp == 0) {
     if (lane == 0) {
-      mbar_arrive_expect_tx(bar(C::BAR_QD), 2 * C::Q_BYTES);
+      if (!C::A_TMEM) {
+        mbar_arrive_expect_tx(bar(C::BAR_QD), 2 * C::Q_BYTES);
 #pragma unroll
-      for (int c = 0; c < C::KCH; ++c) {
-        tma_load_4d(sbase + C::OFF_Q + c * C::Q_CHUNK, &tm_q, bar(C::BAR_QD), c * 64, head0, t0, b);
-        tma_load_4d(sbase + C::OFF_DO + c * C::Q_CHUNK, &tm_do, bar(C::BAR_QD), c * 64, head0, t0, b);
+        for (int c = 0; c < C::KCH; ++c) {
+          tma_load_4d(sbase + C::OFF_Q + c * C::Q_CHUNK, &tm_q, bar(C::BAR_QD), c * 64, head0, t0, b);
+          tma_load_4d(sbase + C::OFF_DO + c * C::Q_CHUNK, &tm_do, bar(C::BAR_QD), c * 64, head0, t0, b);
+        }
       }
       int filled = 0;
       for (int j = 0; j < n_kv; ++j) {
@@ -447,12 +508,13 @@ __global__ void __launch_bounds__(384, 1)
       }
       volatile int zero = 0;
       WaitCtl drain{&zero, p.status, drain_limit_ns(p.timeout_ns)};
-      mbar_wait(bar(C::BAR_QD), 0, drain);
+      if (!C::A_TMEM) mbar_wait(bar(C::BAR_QD), 0, drain);
       for (int j = max(0, filled - C::STAGES); j < filled; ++j)
         mbar_wait(bar(C::BAR_FULL + j % C::STAGES), (j / C::STAGES) & 1, drain);
     }
-  } else if (warp == 1) {
+  } else if (warp == 1 || warp == 3) {
     if (lane == 0) {
+      const int me = warp == 1 ? 0 : 1;
       constexpr uint32_t IDESC_S = idesc_bf16_f32(128, C::BK, 0, 0);
       constexpr uint32_t IDESC_G = idesc_bf16_f32(128, D, 0, 1);
       // descriptors built once; offsets added as o >> 4 (see the dK/dV kernel)
@@ -469,19 +531,24 @@ __global__ void __launch_bounds__(384, 1)
         const uint32_t buf = tmem + (uint32_t)(j & 1) * 128;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint64_t oq = ((kk >> 2) * C::Q_CHUNK + (kk & 3) * 32) >> 4;
           const uint64_t ok_ = ((kk >> 2) * C::T_CHUNK + (kk & 3) * 32) >> 4;
-          umma_ss(buf, dQ + oq, dKk + so + ok_, IDESC_S, kk > 0);
-          umma_ss(buf + 64, dO + oq, dVk + so + ok_, IDESC_S, kk > 0);
+          if (C::A_TMEM) {
+            umma_ts(buf, tmem + C::COL_QT + kk * 8, dKk + so + ok_, IDESC_S, kk > 0);
+            umma_ts(buf + 64, tmem + C::COL_DOT + kk * 8, dVk + so + ok_, IDESC_S, kk > 0);
+          } else {
+            const uint64_t oq = ((kk >> 2) * C::Q_CHUNK + (kk & 3) * 32) >> 4;
+            umma_ss(buf, dQ + oq, dKk + so + ok_, IDESC_S, kk > 0);
+            umma_ss(buf + 64, dO + oq, dVk + so + ok_, IDESC_S, kk > 0);
+          }
         }
         umma_commit(bar(C::BAR_S + (j & 1)));
         return true;
       };
       bool ok = mbar_wait(bar(C::BAR_QD), 0, ctl);
-      if (ok) ok = issue_scores(0);
-      if (ok && n_kv > 1) ok = issue_scores(1);
-      for (int j = 0; ok && j < n_kv; ++j) {
-        if (!mbar_wait(bar(C::BAR_P + (j & 1)), (j >> 1) & 1, ctl)) { ok = false; break; }
+      if (ok && me < n_kv) ok = issue_scores(me);
+      const uint32_t col_dq = tmem + C::COL_DQ + (uint32_t)me * D;
+      for (int j = me; ok && j < n_kv; j += 2) {
+        if (!mbar_wait_spin(bar(C::BAR_P + (j & 1)), (j >> 1) & 1, ctl)) { ok = false; break; }
         tc_fence_after();
         const int st = j % C::STAGES;
         const uint64_t so = (uint64_t)(st * (C::STAGE_BYTES >> 4));
@@ -489,16 +556,16 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
         for (int kk = 0; kk < C::BK / 16; ++kk)
           // dQ += dS K_j (K as an MN-major B operand: d contiguous)
-          umma_ts(tmem + C::COL_DQ, buf + kk * 8, dKm + so + (uint64_t)((kk * 16 * 128) >> 4), IDESC_G,
-                  (j > 0 || kk > 0) ? 1u : 0u);
+          umma_ts(col_dq, buf + kk * 8, dKm + so + (uint64_t)((kk * 16 * 128) >> 4), IDESC_G,
+                  (j > me || kk > 0) ? 1u : 0u);
         umma_commit(bar(C::BAR_EMPTY + st));
         if (j + 2 < n_kv) ok = issue_scores(j + 2);
       }
-      if (ok) umma_commit(bar(C::BAR_DONE));
-      umma_commit(bar(C::BAR_DRAIN));
+      if (ok) umma_commit(bar(C::BAR_DONE + me));
+      umma_commit(bar(C::BAR_DRAIN + me));
       volatile int zero = 0;
       WaitCtl drain{&zero, p.status, drain_limit_ns(p.timeout_ns)};
-      mbar_wait(bar(C::BAR_DRAIN), 0, drain);
+      mbar_wait(bar(C::BAR_DRAIN + me), 0, drain);
     }
   } else if (warp >= 4) {
     const int wg = (warp - 4) >> 2;
@@ -510,55 +577,88 @@ __global__ void __launch_bounds__(384, 1)
     const uint32_t lane_base = tmem + (uint32_t(quarter * 32) << 16);
     const uint32_t buf = lane_base + (uint32_t)wg * 128;
     const float sl2 = p.scale_log2;
-    float lse2_r = 0.f, dsum_r = 0.f;
+    float nl_r = 0.f, nd_r = 0.f;
     if (row_ok) {
       const size_t ri = ((size_t)b * p.H_q + head) * p.ld + token;
-      lse2_r = p.lse2[ri];
-      dsum_r = p.dsum[ri];
+      nl_r = p.nlse2[ri];
+      nd_r = p.ndsum[ri];
+    }
+    if (C::A_TMEM) {
+      // this row of Q (warpgroup 0) or dO (warpgroup 1) into the TMEM lane
+      const __nv_bfloat16* src = (wg == 0 ? p.q : p.dout) + (((size_t)b * p.N + (row_ok ? token : 0)) * p.H_q + head) * D;
+      uint32_t r[32];
+      const uint4* s4 = reinterpret_cast<const uint4*>(src);
+#pragma unroll
+      for (int x = 0; x < 8; ++x) {
+        const uint4 a = row_ok ? s4[x] : make_uint4(0u, 0u, 0u, 0u);
+        r[4 * x] = a.x; r[4 * x + 1] = a.y; r[4 * x + 2] = a.z; r[4 * x + 3] = a.w;
+      }
+      tmem_st32(lane_base + (wg == 0 ? C::COL_QT : C::COL_DOT), r);
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(C::BAR_QD));
+    }
+    float2 nl[8], nd[8];
+#pragma unroll
+    for (int w = 0; w < 8; ++w) {
+      nl[w] = make_float2(nl_r, nl_r);
+      nd[w] = make_float2(nd_r, nd_r);
     }
     bool ok = true;
     for (int j = wg; j < n_kv; j += 2) {
-      if (!mbar_wait_warp(bar(C::BAR_S + wg), (j >> 1) & 1, ctl)) { ok = false; break; }
+      // the warpgroups take turns (see the dK/dV kernel)
+      if (!mbar_wait_warp(bar(C::BAR_S + wg), (j >> 1) & 1, ctl) ||
+          (j > 0 && !mbar_wait_warp(bar(C::BAR_P + (wg ^ 1)), ((j - 1) >> 1) & 1, ctl))) {
+        ok = false;
+        break;
+      }
       tc_fence_after();
       // keys above t0 only in the last tiles when causal; keys past N in the last tile
       const bool need_mask = !row_ok || (j * C::BK + C::BK > p.N) || (p.causal && j * C::BK + C::BK - 1 > t0);
+      uint32_t a0[16], b0[16], a1[16], b1[16];
+      tmem_ld16x2_nowait(buf, buf + 64, a0, b0);
+      tmem_ld_wait16x2(a0, b0);
 #pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        uint32_t rs[32], rd[32];
-        tmem_ld32x2(buf + c * 32, buf + 64 + c * 32, rs, rd);
+      for (int k = 0; k < 4; ++k) {
+        uint32_t(&ra)[16] = (k & 1) ? a1 : a0;
+        uint32_t(&rb)[16] = (k & 1) ? b1 : b0;
+        uint32_t(&na)[16] = (k & 1) ? a0 : a1;
+        uint32_t(&nb)[16] = (k & 1) ? b0 : b1;
+        if (k < 3) tmem_ld16x2_nowait(buf + 16 * (k + 1), buf + 64 + 16 * (k + 1), na, nb);
         if (need_mask) {   // masked scores -> -inf (p = 0), outside the arithmetic block
 #pragma unroll
-          for (int x = 0; x < 32; ++x) {
-            const int key = j * C::BK + c * 32 + x;
-            if (!row_ok || key >= p.N || (p.causal && key > token)) rs[x] = __float_as_uint(-INFINITY);
+          for (int x = 0; x < 16; ++x) {
+            const int key = j * C::BK + k * 16 + x;
+            if (!row_ok || key >= p.N || (p.causal && key > token)) ra[x] = __float_as_uint(-INFINITY);
           }
         }
-        uint32_t pd[16];
-#pragma unroll
-        for (int w = 0; w < 16; ++w) {
-          float dv[2];
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const float pe = ex2_approx(fmaf(__uint_as_float(rs[2 * w + h]), sl2, -lse2_r));
-            dv[h] = pe * (__uint_as_float(rd[2 * w + h]) - dsum_r);
-          }
-          pd[w] = pack_bf16x2(dv[0], dv[1]);
-        }
-        tmem_st16(buf + c * 16, pd);
+        uint32_t pp[8], pd[8];
+        bwd_chunk(ra, rb, sl2, nl, nd, pp, pd);
+        tmem_st8(buf + k * 8, pd);
+        if (k < 3) tmem_ld_wait16x2(na, nb);
       }
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(C::BAR_P + wg));
     }
-    // epilogue: each warpgroup writes half of the row's d columns (x scale)
-    if (ok && mbar_wait_warp(bar(C::BAR_DONE), 0, ctl)) {
+    // epilogue: each warpgroup writes half of the row's d columns (x scale),
+    // the sum of the two issuers' accumulators
+    const bool two = n_kv > 1;
+    if (ok && mbar_wait_warp(bar(C::BAR_DONE), 0, ctl) && (!two || mbar_wait_warp(bar(C::BAR_DONE + 1), 0, ctl))) {
       tc_fence_after();
       __nv_bfloat16* dst = p.dq + (((size_t)b * p.N + (row_ok ? token : 0)) * p.H_q + head) * D;
 #pragma unroll
       for (int c = wg * (D / 2); c < (wg + 1) * (D / 2); c += 32) {
-        uint32_t r[32];
-        tmem_ld32(lane_base + C::COL_DQ + c, r);
+        uint32_t r[32], r1[32];
+        if (two) {
+          tmem_ld32x2(lane_base + C::COL_DQ + c, lane_base + C::COL_DQ + D + c, r, r1);
+#pragma unroll
+          for (int x = 0; x < 32; ++x) r[x] = __float_as_uint(__uint_as_float(r[x]) + __uint_as_float(r1[x]));
+        } else {
+          tmem_ld32(lane_base + C::COL_DQ + c, r);
+        }
         uint4 w[4];
         uint32_t* wp = reinterpret_cast<uint32_t*>(w);
 #pragma unroll

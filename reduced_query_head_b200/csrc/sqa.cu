@@ -340,11 +340,15 @@ int launch_attn_bwd(const DeviceState* st, const void* q, const void* k, const v
   if (int e = encode_rows_f32(&td, dsum, (long long)B * H_q, N, ld, DkdvCfg<D>::BQ)) return e;
 
   BwdParams p;
+  p.q = reinterpret_cast<const __nv_bfloat16*>(q);
+  p.k = reinterpret_cast<const __nv_bfloat16*>(k);
+  p.v = reinterpret_cast<const __nv_bfloat16*>(v);
+  p.dout = reinterpret_cast<const __nv_bfloat16*>(dout);
   p.dq = reinterpret_cast<__nv_bfloat16*>(dq);
   p.dk = reinterpret_cast<__nv_bfloat16*>(dk);
   p.dv = reinterpret_cast<__nv_bfloat16*>(dv);
-  p.lse2 = lse2;
-  p.dsum = dsum;
+  p.nlse2 = lse2;
+  p.ndsum = dsum;
   p.ld = ld;
   p.B = B;
   p.N = N;
