@@ -338,8 +338,10 @@ __global__ void __launch_bounds__(384, 1)
         const bool more = j + 1 < nk;
         {
           // S(j+1) as soon as the softmax has read S(j): overlaps softmax(j).
+          // This thread spins on its hand-offs (a suspended wait wakes a few
+          // hundred cycles after the phase completes).
           if (more) {
-            if (!mbar_wait(bar(C::BAR_SFREE + k), j & 1, ctl) || !mbar_wait(bar(C::BAR_KF + s1), ph1, ctl)) {
+            if (!mbar_wait_spin(bar(C::BAR_SFREE + k), j & 1, ctl) || !mbar_wait(bar(C::BAR_KF + s1), ph1, ctl)) {
               ok = false;
               break;
             }
@@ -348,7 +350,7 @@ __global__ void __launch_bounds__(384, 1)
             umma_commit(bar(C::BAR_S + k));
           }
         }
-        if (!mbar_wait(bar(C::BAR_VF + s), ph, ctl) || !mbar_wait(bar(C::BAR_P + k), j & 1, ctl)) {
+        if (!mbar_wait(bar(C::BAR_VF + s), ph, ctl) || !mbar_wait_spin(bar(C::BAR_P + k), j & 1, ctl)) {
           ok = false;
           break;
         }
