@@ -39,12 +39,12 @@ L2_FLUSH_BYTES = 256 << 20     # > 126 MB L2
 
 
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "attn_traffic_headcfg32k.json")
-KERNEL_SOURCES = ["attn_fwd.cuh", "sm100.cuh", "sqa.cu"]
+KERNEL_SOURCES = ["attn_fwd.cuh", "sm100.cuh"]
 
 
 def kernel_source_hash():
-    """sha256 over the attention kernel's sources: DRAM counters taken from an
-    older build of the kernel are not reported against a newer one."""
+    """sha256 over the forward attention kernel's device sources: DRAM counters
+    taken from an older build of the kernel are not reported against a newer one."""
     import hashlib
     h = hashlib.sha256()
     for name in KERNEL_SOURCES:
