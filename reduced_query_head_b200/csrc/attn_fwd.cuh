@@ -231,26 +231,30 @@ __global__ void __launch_bounds__(384, 1)
     if (lane == 0) {
       constexpr uint32_t IDESC_S = idesc_bf16_f32(C::BM, C::BN, 0, 0);
       constexpr uint32_t IDESC_O = idesc_bf16_f32(C::BM, D, 0, 1);
+      // Descriptors are built once; a byte offset o inside shared memory is
+      // added as o >> 4 to the start-address field (no carry: smem < 256 KB).
+      const uint64_t dq0 = sdesc_sw128(sbase + C::OFF_Q, 16, 1024);
+      const uint64_t dk0 = sdesc_sw128(sbase + C::OFF_K, 16, 1024);
+      const uint64_t dv0 = sdesc_sw128(sbase + C::OFF_V, C::CHUNK_KV, 1024);
       auto issue_s = [&](int k, int s) {
-        const uint32_t qa = sbase + C::OFF_Q + k * C::Q_BYTES;
-        const uint32_t ka = sbase + C::OFF_K + s * C::KV_BYTES;
+        const uint64_t dq = dq0 + (uint64_t)((k * C::Q_BYTES) >> 4);
+        const uint64_t dk = dk0 + (uint64_t)((s * C::KV_BYTES) >> 4);
         const uint32_t col_s = k ? C::COL_S1 : C::COL_S0;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * C::CHUNK_Q + (kk & 3) * 32;
-          const uint32_t offk = (kk >> 2) * C::CHUNK_KV + (kk & 3) * 32;
-          umma_ss(tmem + col_s, sdesc_sw128(qa + off, 16, 1024), sdesc_sw128(ka + offk, 16, 1024), IDESC_S,
-                  kk > 0);
+          const uint64_t off = ((kk >> 2) * C::CHUNK_Q + (kk & 3) * 32) >> 4;
+          const uint64_t offk = ((kk >> 2) * C::CHUNK_KV + (kk & 3) * 32) >> 4;
+          umma_ss(tmem + col_s, dq + off, dk + offk, IDESC_S, kk > 0);
         }
       };
       auto issue_pv = [&](int k, int s, int j) {
-        const uint32_t va = sbase + C::OFF_V + s * C::KV_BYTES;
+        const uint64_t dv = dv0 + (uint64_t)((s * C::KV_BYTES) >> 4);
         const uint32_t col_o = k ? C::COL_O1 : C::COL_O0;
         const uint32_t col_p = k ? C::COL_P1 : C::COL_P0;
 #pragma unroll
         for (int kk = 0; kk < C::BN / 16; ++kk) {
-          umma_ts(tmem + col_o, tmem + col_p + kk * 8, sdesc_sw128(va + kk * 16 * 128, C::CHUNK_KV, 1024),
-                  IDESC_O, (j > 0 || kk > 0) ? 1u : 0u);
+          umma_ts(tmem + col_o, tmem + col_p + kk * 8, dv + (uint64_t)((kk * 16 * 128) >> 4), IDESC_O,
+                  (j > 0 || kk > 0) ? 1u : 0u);
         }
       };
       bool ok = n_max > 0 && mbar_wait(bar(C::BAR_Q), 0, ctl) && mbar_wait(bar(C::BAR_KF + 0), 0, ctl);
@@ -304,24 +308,26 @@ __global__ void __launch_bounds__(384, 1)
       const uint32_t col_s = k ? C::COL_S1 : C::COL_S0;
       const uint32_t col_o = k ? C::COL_O1 : C::COL_O0;
       const uint32_t col_p = k ? C::COL_P1 : C::COL_P0;
-      const uint32_t qa = sbase + C::OFF_Q + k * C::Q_BYTES;
       const int nk = n_kv[k];
+      // descriptors built once; offsets added as o >> 4 (see the D = 128 path)
+      const uint64_t dq = sdesc_sw128(sbase + C::OFF_Q + k * C::Q_BYTES, 16, 1024);
+      const uint64_t dk0 = sdesc_sw128(sbase + C::OFF_K, 16, 1024);
+      const uint64_t dv0 = sdesc_sw128(sbase + C::OFF_V, C::CHUNK_KV, 1024);
       auto issue_s = [&](int s) {
-        const uint32_t ka = sbase + C::OFF_K + s * C::KV_BYTES;
+        const uint64_t dk = dk0 + (uint64_t)((s * C::KV_BYTES) >> 4);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * C::CHUNK_Q + (kk & 3) * 32;
-          const uint32_t offk = (kk >> 2) * C::CHUNK_KV + (kk & 3) * 32;
-          umma_ss(tmem + col_s, sdesc_sw128(qa + off, 16, 1024), sdesc_sw128(ka + offk, 16, 1024), IDESC_S,
-                  kk > 0);
+          const uint64_t off = ((kk >> 2) * C::CHUNK_Q + (kk & 3) * 32) >> 4;
+          const uint64_t offk = ((kk >> 2) * C::CHUNK_KV + (kk & 3) * 32) >> 4;
+          umma_ss(tmem + col_s, dq + off, dk + offk, IDESC_S, kk > 0);
         }
       };
       auto issue_pv = [&](int s, int j) {
-        const uint32_t va = sbase + C::OFF_V + s * C::KV_BYTES;
+        const uint64_t dv = dv0 + (uint64_t)((s * C::KV_BYTES) >> 4);
 #pragma unroll
         for (int kk = 0; kk < C::BN / 16; ++kk) {
-          umma_ts(tmem + col_o, tmem + col_p + kk * 8, sdesc_sw128(va + kk * 16 * 128, C::CHUNK_KV, 1024),
-                  IDESC_O, (j > 0 || kk > 0) ? 1u : 0u);
+          umma_ts(tmem + col_o, tmem + col_p + kk * 8, dv + (uint64_t)((kk * 16 * 128) >> 4), IDESC_O,
+                  (j > 0 || kk > 0) ? 1u : 0u);
         }
       };
       bool ok = nk > 0 && mbar_wait(bar(C::BAR_Q), 0, ctl) && mbar_wait(bar(C::BAR_KF + 0), 0, ctl);

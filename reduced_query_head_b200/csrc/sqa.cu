@@ -59,7 +59,7 @@ AttnKernel attn_kernel_128(int i) {
   return t[i];
 }
 // Default split per head size; SQA_EXP2_POLY_EIGHTHS=<0|2|3|4|5> overrides it.
-constexpr int kDefaultEmu64 = 2, kDefaultEmu128 = 2;
+constexpr int kDefaultEmu64 = 0, kDefaultEmu128 = 2;
 int emu_index(int d) {
   int want = d == 64 ? kDefaultEmu64 : kDefaultEmu128;
   if (const char* e = getenv("SQA_EXP2_POLY_EIGHTHS")) {
