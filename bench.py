@@ -371,9 +371,11 @@ def oracle_sample(rows_per_cfg, seed=0):
 
 
 def cpu_baseline(seconds=15.0):
-    # size the sample from a short probe so the whole leg takes ~`seconds`
-    f0, s0 = oracle_sample(8)
-    rows = int(max(8, min(4096, 8 * seconds / max(s0, 1e-3))))
+    # size the sample from a probe taken after a warm-up call (thread pool,
+    # first-touch allocation), so the whole leg takes about `seconds`
+    oracle_sample(8)
+    f1, s1 = oracle_sample(64)
+    rows = int(max(64, min(8192, 64 * seconds / max(s1, 1e-3))))
     f, s = oracle_sample(rows)
     return {"value": round(f / s / 1e12, 6), "unit": "TFLOP/s", "cores": _blas_threads(), "kind": "oracle",
             "sample": "%d query positions (all heads) of each of the 7 head configs at N=32768, d=64, "

@@ -44,21 +44,21 @@ struct DeviceState {
 // Attention kernels by the share of exp2 evaluated on the FMA pipe (eighths
 // of the column pairs; the rest use the MUFU unit).
 using AttnKernel = void (*)(const CUtensorMap, const CUtensorMap, const CUtensorMap, const AttnParams);
-constexpr int kEmuChoices[] = {0, 2, 3, 4, 5};
-constexpr int kNumEmu = 5;
+constexpr int kEmuChoices[] = {0, 1, 2, 3, 4, 5};
+constexpr int kNumEmu = 6;
 AttnKernel attn_kernel_64(int i) {
-  static const AttnKernel t[kNumEmu] = {sqa::attn_fwd_kernel<64, 0>, sqa::attn_fwd_kernel<64, 2>,
-                                        sqa::attn_fwd_kernel<64, 3>, sqa::attn_fwd_kernel<64, 4>,
-                                        sqa::attn_fwd_kernel<64, 5>};
+  static const AttnKernel t[kNumEmu] = {sqa::attn_fwd_kernel<64, 0>, sqa::attn_fwd_kernel<64, 1>,
+                                        sqa::attn_fwd_kernel<64, 2>, sqa::attn_fwd_kernel<64, 3>,
+                                        sqa::attn_fwd_kernel<64, 4>, sqa::attn_fwd_kernel<64, 5>};
   return t[i];
 }
 AttnKernel attn_kernel_128(int i) {
-  static const AttnKernel t[kNumEmu] = {sqa::attn_fwd_kernel<128, 0>, sqa::attn_fwd_kernel<128, 2>,
-                                        sqa::attn_fwd_kernel<128, 3>, sqa::attn_fwd_kernel<128, 4>,
-                                        sqa::attn_fwd_kernel<128, 5>};
+  static const AttnKernel t[kNumEmu] = {sqa::attn_fwd_kernel<128, 0>, sqa::attn_fwd_kernel<128, 1>,
+                                        sqa::attn_fwd_kernel<128, 2>, sqa::attn_fwd_kernel<128, 3>,
+                                        sqa::attn_fwd_kernel<128, 4>, sqa::attn_fwd_kernel<128, 5>};
   return t[i];
 }
-// Default split per head size; SQA_EXP2_POLY_EIGHTHS=<0|2|3|4|5> overrides it.
+// Default split per head size; SQA_EXP2_POLY_EIGHTHS=<0..5> overrides it.
 constexpr int kDefaultEmu64 = 0, kDefaultEmu128 = 2;
 int emu_index(int d) {
   int want = d == 64 ? kDefaultEmu64 : kDefaultEmu128;
