@@ -388,3 +388,31 @@ def attention_backward_bound(q, k, v, dout, causal: bool, scale: float):
             ek[b, :, g, :] += bk
             ev[b, :, g, :] += bv
     return eq, ek, ev
+
+
+# ---------------------------------------------------------------------------
+# Decode: one new token per sequence attends to its whole key/value cache.
+#
+# The GQA explainer's motivation is the autoregressive step ("背景と動機", the
+# KV-cache table): each step reads the cache of H_kv groups, and every query
+# head of a group reads the same cached K/V. The new token sits at the end of
+# the cache (its own K/V already appended), so it sees every cached key: the
+# last row of causal attention over the cache.
+# ---------------------------------------------------------------------------
+
+def decode(q, k_cache, v_cache, scale: float) -> np.ndarray:
+    """out [B, H_q, d] for q [B, H_q, d] against k_cache/v_cache [B, N, H_kv, d] (float64)."""
+    q = np.asarray(q, dtype=np.float64)
+    k_cache = np.asarray(k_cache, dtype=np.float64)
+    v_cache = np.asarray(v_cache, dtype=np.float64)
+    B, H_q, d = q.shape
+    H_kv = k_cache.shape[2]
+    out = np.empty_like(q)
+    for b in range(B):
+        for i in range(H_q):
+            g = group_of_head(i, H_q, H_kv)
+            kh = np.array(k_cache[b, :, g, :])     # explicit repetition: head i's own copy
+            vh = np.array(v_cache[b, :, g, :])
+            s = scale * (kh @ q[b, i, :])           # explicit score row over all cached keys
+            out[b, i, :] = _softmax_rows_times_v(s[None, :], vh)[0]
+    return out

@@ -290,3 +290,43 @@ def test_planted_missing_normalisation_is_caught(monkeypatch):
                         lambda s, vh: np.exp(s - s.max(1, keepdims=True)) @ vh)
     with pytest.raises(AssertionError):
         test_zero_query_gives_mean_of_values(8, 2)
+
+
+# ---------------------------------------------------------------- decode
+@pytest.mark.parametrize("H_q,H_kv", [(4, 4), (8, 2), (6, 4), (16, 1)])
+def test_decode_is_last_causal_row(H_q, H_kv):
+    # the new token at position N-1 sees every cached key: the last row of causal attention
+    rng = np.random.default_rng(50)
+    B, N, d, scale = 2, 37, 8, 0.3
+    q = rng.standard_normal((B, N, H_q, d))
+    k, v = rng.standard_normal((B, N, H_kv, d)), rng.standard_normal((B, N, H_kv, d))
+    want = oracle.attention(q, k, v, True, scale)[:, N - 1]
+    got = oracle.decode(q[:, N - 1], k, v, scale)
+    np.testing.assert_allclose(got, want, rtol=0, atol=1e-13)
+
+
+def test_decode_closed_forms():
+    rng = np.random.default_rng(51)
+    B, N, H_q, H_kv, d = 1, 9, 4, 2, 5
+    k, v = rng.standard_normal((B, N, H_kv, d)), rng.standard_normal((B, N, H_kv, d))
+    # q = 0: uniform weights, the mean of the group's cached values
+    out = oracle.decode(np.zeros((B, H_q, d)), k, v, 0.7)
+    for i in range(H_q):
+        np.testing.assert_allclose(out[0, i], v[0, :, (i * H_kv) // H_q].mean(axis=0), atol=1e-14)
+    # one cached key: its value, whatever the query
+    out1 = oracle.decode(rng.standard_normal((B, H_q, d)), k[:, :1], v[:, :1], 0.7)
+    for i in range(H_q):
+        np.testing.assert_allclose(out1[0, i], v[0, 0, (i * H_kv) // H_q], atol=0)
+
+
+def test_decode_against_torch_sdpa():
+    rng = np.random.default_rng(52)
+    B, N, H_q, H_kv, d, scale = 2, 23, 8, 2, 16, 0.25
+    q = rng.standard_normal((B, H_q, d))
+    k, v = rng.standard_normal((B, N, H_kv, d)), rng.standard_normal((B, N, H_kv, d))
+    R = H_q // H_kv
+    tq = torch.from_numpy(q)[:, :, None, :]
+    tk = torch.from_numpy(k).permute(0, 2, 1, 3).repeat_interleave(R, dim=1)
+    tv = torch.from_numpy(v).permute(0, 2, 1, 3).repeat_interleave(R, dim=1)
+    want = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv, scale=scale)[:, :, 0].numpy()
+    np.testing.assert_allclose(oracle.decode(q, k, v, scale), want, atol=1e-12)
