@@ -585,6 +585,35 @@ def _bench_extra(args, sqa, torch, device, stream, flush, peaks, lines):
                           "pct_of_peak": round(100 * fl / (med * 1e-3) / 1e12 / peaks["bf16_tflops"], 1)})
             print(json.dumps(lines[-1]), flush=True)
             del dev, out, lse, ws, dq, dk, dv, do
+    elif args.workload == "decode":
+        # one new token per sequence against a 32768-token cache, the headline's head configurations;
+        # memory-bound: bytes = the K/V cache (+ q and out), against the measured HBM copy bandwidth
+        import synth
+        B, N, d = args.B, args.N, args.d
+        for name, H_q, H_kv in HEAD_CONFIGS_32K:
+            def mk(shape, tensor):
+                h = torch.empty(shape, dtype=torch.bfloat16)
+                synth.fill_bf16_into(h.data_ptr(), h.numel(), 0, tensor, 1.0)
+                return h.to(device)
+            q, k, v = mk((B, H_q, d), "q"), mk((B, N, H_kv, d), "k"), mk((B, N, H_kv, d), "v")
+            out = torch.empty((B, H_q, d), dtype=torch.bfloat16, device=device)
+            ws_bytes = sqa.sqa_decode_workspace_bytes(B, N, H_q, H_kv, d)
+            ws = torch.empty(ws_bytes, dtype=torch.uint8, device=device)
+
+            def fn():
+                sqa.sqa_decode_fwd(q, k, v, out, ws, ws_bytes, B, N, H_q, H_kv, d, d ** -0.5, stream)
+            for _ in range(args.warmup):
+                fn()
+            ms = _time_launches(fn, args.steps, flush, stream)
+            assert sqa.sqa_device_status(stream) == 0
+            med = statistics.median(ms)
+            nbytes = 2.0 * B * N * H_kv * d * 2 + 2.0 * 2 * B * H_q * d
+            gbs = nbytes / (med * 1e-3) / 1e9
+            lines.append({"workload": "decode", "config": name, "B": B, "N": N, "H_q": H_q, "H_kv": H_kv, "d": d,
+                          "us_median": round(med * 1e3, 2), "GB_per_s": round(gbs, 1),
+                          "frac_of_hbm": round(gbs / peaks["hbm_gbs"], 3), "bytes": int(nbytes)})
+            print(json.dumps(lines[-1]), flush=True)
+            del q, k, v, out, ws
     elif args.workload == "layer":
         import synth
         B, N, dm, H_q, H_kv, d = 4, 16384, 2048, 16, 8, 64
@@ -634,9 +663,10 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["sqa", "reference"], default="sqa")
-    ap.add_argument("--workload", choices=["headcfg32k", "small", "long", "layer", "sweep", "single", "linear", "bwd"],
+    ap.add_argument("--workload", choices=["headcfg32k", "small", "long", "layer", "sweep", "single", "linear", "bwd", "decode"],
                     default="headcfg32k")
     ap.add_argument("--N", type=int, default=32768)
+    ap.add_argument("--B", type=int, default=8, help="sequences per decode step (--workload decode)")
     ap.add_argument("--hq", type=int, default=16)
     ap.add_argument("--hkv", type=int, default=16)
     ap.add_argument("--d", type=int, default=64)

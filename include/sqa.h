@@ -107,6 +107,34 @@ int sqa_attn_bwd(const void* q, const void* k, const void* v, const void* out, c
                  int causal, float scale, void* stream);
 
 /*
+ * Bytes of device workspace sqa_decode_fwd needs (fp32 partial results of
+ * the split key ranges). Returns 0 for invalid sizes.
+ */
+size_t sqa_decode_workspace_bytes(int B, int N, int H_q, int H_kv, int d_head);
+
+/*
+ * Decode step: one new token per sequence attends to its whole K/V cache
+ * (the autoregressive step the GQA explainer motivates, "背景と動機" and its
+ * KV-cache table; every query head of a group reads the same cached K/V):
+ *   out[b,i,:] = sum_u softmax_u(scale * q[b,i,:] . k_cache[b,u,g(i),:]) v_cache[b,u,g(i),:]
+ * over all u in [0, N), g(i) = floor(i * H_kv / H_q). The new token's own K/V
+ * are expected to be in the cache already (it is the last row of causal
+ * attention over the cache).
+ *   q        [B, H_q, d_head] bf16
+ *   k_cache  [B, N, H_kv, d_head] bf16 (the layout of sqa_attn_fwd's k)
+ *   v_cache  [B, N, H_kv, d_head] bf16
+ *   out      [B, H_q, d_head] bf16, written in full
+ *   workspace: device memory of at least sqa_decode_workspace_bytes(...),
+ *              256-byte aligned; scratch, overwritten.
+ * Requirements: B, N >= 1; 1 <= H_kv <= H_q; d_head in {64, 128}; scale
+ * finite and > 0. Arithmetic: bf16 inputs, fp32 scores, softmax and sums, P
+ * rounded to bf16 for the P.V product, bf16 output.
+ */
+int sqa_decode_fwd(const void* q, const void* k_cache, const void* v_cache, void* out,
+                   void* workspace, size_t workspace_bytes,
+                   int B, int N, int H_q, int H_kv, int d_head, float scale, void* stream);
+
+/*
  * Bytes of device workspace sqa_layer_fwd needs (Q, K, V and the merged
  * attention output, each 256-byte aligned). Returns 0 for invalid sizes.
  */

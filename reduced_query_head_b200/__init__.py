@@ -15,7 +15,7 @@ from .build import LIB as _LIB_PATH
 __all__ = [
     "SQA_OK", "SQA_ERR_INVALID_ARG", "SQA_ERR_UNSUPPORTED", "SQA_ERR_CUDA", "SQA_ERR_TIMEOUT",
     "SQA_ERR_WORKSPACE", "SqaError", "lib", "EXPORTED_SYMBOLS", "sqa_attn_fwd", "sqa_attn_fwd_lse",
-    "sqa_attn_bwd_workspace_bytes", "sqa_attn_bwd", "sqa_layer_fwd",
+    "sqa_attn_bwd_workspace_bytes", "sqa_attn_bwd", "sqa_decode_workspace_bytes", "sqa_decode_fwd", "sqa_layer_fwd",
     "sqa_layer_workspace_bytes", "sqa_layer_fwd_static_ws", "SQA_STATIC_WORKSPACE_BYTES", "sqa_linear_fwd",
     "sqa_device_status", "sqa_set_wait_limit_ns",
     "sqa_check_wait_timeout", "sqa_status_string", "sqa_version",
@@ -25,7 +25,8 @@ SQA_OK, SQA_ERR_INVALID_ARG, SQA_ERR_UNSUPPORTED, SQA_ERR_CUDA, SQA_ERR_TIMEOUT,
 SQA_STATIC_WORKSPACE_BYTES = 64 << 20   # include/sqa.h
 
 EXPORTED_SYMBOLS = (
-    "sqa_attn_fwd", "sqa_attn_fwd_lse", "sqa_attn_bwd_workspace_bytes", "sqa_attn_bwd", "sqa_layer_workspace_bytes", "sqa_layer_fwd", "sqa_layer_fwd_static_ws", "sqa_linear_fwd",
+    "sqa_attn_fwd", "sqa_attn_fwd_lse", "sqa_attn_bwd_workspace_bytes", "sqa_attn_bwd",
+    "sqa_decode_workspace_bytes", "sqa_decode_fwd", "sqa_layer_workspace_bytes", "sqa_layer_fwd", "sqa_layer_fwd_static_ws", "sqa_linear_fwd",
     "sqa_device_status",
     "sqa_set_wait_limit_ns", "sqa_check_wait_timeout", "sqa_status_string", "sqa_version",
 )
@@ -46,6 +47,10 @@ lib.sqa_attn_bwd_workspace_bytes.argtypes = [_i, _i, _i]
 lib.sqa_attn_bwd_workspace_bytes.restype = _sz
 lib.sqa_attn_bwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _i, _i, _i, _i, _i, _i, _f, _vp]
 lib.sqa_attn_bwd.restype = _i
+lib.sqa_decode_workspace_bytes.argtypes = [_i, _i, _i, _i, _i]
+lib.sqa_decode_workspace_bytes.restype = _sz
+lib.sqa_decode_fwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _sz, _i, _i, _i, _i, _i, _f, _vp]
+lib.sqa_decode_fwd.restype = _i
 lib.sqa_layer_workspace_bytes.argtypes = [_i, _i, _i, _i, _i, _i]
 lib.sqa_layer_workspace_bytes.restype = _sz
 lib.sqa_layer_fwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _i, _i, _i, _i, _i, _i, _i, _f, _vp]
@@ -123,6 +128,18 @@ def sqa_attn_bwd(q, k, v, out, dout, lse, dq, dk, dv, workspace, workspace_bytes
                           _ptr(dv), _ptr(workspace), int(workspace_bytes), B, N, H_q, H_kv, d_head, int(causal),
                           float(scale), _stream(stream))
     return _check(st, "sqa_attn_bwd", raise_on_error)
+
+
+def sqa_decode_workspace_bytes(B, N, H_q, H_kv, d_head):
+    return int(lib.sqa_decode_workspace_bytes(B, N, H_q, H_kv, d_head))
+
+
+def sqa_decode_fwd(q, k_cache, v_cache, out, workspace, workspace_bytes, B, N, H_q, H_kv, d_head, scale,
+                   stream=None, raise_on_error=True):
+    """One new token per sequence (q [B,H_q,d]) against its K/V cache [B,N,H_kv,d] -> out [B,H_q,d]."""
+    st = lib.sqa_decode_fwd(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(out), _ptr(workspace),
+                            int(workspace_bytes), B, N, H_q, H_kv, d_head, float(scale), _stream(stream))
+    return _check(st, "sqa_decode_fwd", raise_on_error)
 
 
 def sqa_layer_workspace_bytes(B, N, d_model, H_q, H_kv, d_head):

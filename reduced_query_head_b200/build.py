@@ -10,7 +10,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libsqa.so")
 SOURCES = ["sqa.cu"]
-HEADERS = ["sm100.cuh", "attn_fwd.cuh", "attn_bwd.cuh", "gemm.cuh"]
+HEADERS = ["sm100.cuh", "attn_fwd.cuh", "attn_bwd.cuh", "decode.cuh", "gemm.cuh"]
 INCLUDE = os.path.join(ROOT, "include")
 
 NVCC_FLAGS = [

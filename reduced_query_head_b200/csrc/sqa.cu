@@ -13,6 +13,7 @@
 #include "sqa.h"
 #include "attn_bwd.cuh"
 #include "attn_fwd.cuh"
+#include "decode.cuh"
 #include "gemm.cuh"
 
 // Per-device status word written by kernels whose bounded waits ran out.
@@ -23,6 +24,8 @@ namespace {
 using sqa::AttnCfg;
 using sqa::AttnParams;
 using sqa::BwdParams;
+using sqa::DecodeCfg;
+using sqa::DecodeParams;
 using sqa::DkdvCfg;
 using sqa::DqCfg;
 using sqa::GemmCfg;
@@ -119,7 +122,11 @@ int device_state(DeviceState** out) {
         cudaFuncSetAttribute(sqa::bwd_dq_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              DqCfg<64>::SMEM_BYTES) != cudaSuccess ||
         cudaFuncSetAttribute(sqa::bwd_dq_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             DqCfg<128>::SMEM_BYTES) != cudaSuccess)
+                             DqCfg<128>::SMEM_BYTES) != cudaSuccess ||
+        cudaFuncSetAttribute(sqa::decode_split_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             DecodeCfg<64>::SMEM_BYTES) != cudaSuccess ||
+        cudaFuncSetAttribute(sqa::decode_split_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             DecodeCfg<128>::SMEM_BYTES) != cudaSuccess)
       return SQA_ERR_CUDA;
     st.ready = true;
   }
@@ -295,6 +302,67 @@ size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 int bwd_row_ld(int N) { return (N + 3) & ~3; }
 size_t bwd_vec_bytes(int B, int N, int H_q) { return align256((size_t)B * H_q * bwd_row_ld(N) * 4); }
 
+// Decode work split: the keys of each (b, g, head block) are cut into `splits`
+// ranges of whole 64-key tiles, aiming at about four waves of the two resident
+// CTAs on each of 148 SMs (many short CTAs balance the SMs; each still streams
+// several tiles). A pure function of the sizes, so the workspace size is too.
+struct DecodeSplit {
+  int hblocks, splits, tiles_per_split, n_parts, heads_per_cta;
+};
+DecodeSplit decode_split(int B, int N, int H_q, int H_kv, int d) {
+  DecodeSplit r;
+  r.heads_per_cta = 16 * (d == 64 ? DecodeCfg<64>::RB : DecodeCfg<128>::RB);
+  const int r_max = (H_q + H_kv - 1) / H_kv;
+  r.hblocks = (r_max + r.heads_per_cta - 1) / r.heads_per_cta;
+  const int n_tiles = (N + 63) / 64;
+  const long long base = (long long)B * H_kv * r.hblocks;
+  long long want = (4 * 296 + base - 1) / base;
+  if (want < 1) want = 1;
+  if (want > n_tiles) want = n_tiles;
+  r.tiles_per_split = (int)((n_tiles + want - 1) / want);
+  r.splits = (n_tiles + r.tiles_per_split - 1) / r.tiles_per_split;
+  r.n_parts = 4 * r.splits;
+  return r;
+}
+
+template <int D>
+int launch_decode(const DeviceState* st, const void* q, const void* k, const void* v, void* out, void* workspace,
+                  int B, int N, int H_q, int H_kv, float scale, cudaStream_t stream) {
+  using C = DecodeCfg<D>;
+  const DecodeSplit sp = decode_split(B, N, H_q, H_kv, D);
+  if ((long long)B * H_kv > 65535 || sp.hblocks > 65535) return SQA_ERR_INVALID_ARG;
+  CUtensorMap tk, tv;
+  {
+    const cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)H_kv, (cuuint64_t)N, (cuuint64_t)B};
+    const cuuint64_t strides[3] = {(cuuint64_t)D * 2, (cuuint64_t)H_kv * D * 2, (cuuint64_t)N * H_kv * D * 2};
+    const cuuint32_t box[4] = {64, 1, (cuuint32_t)C::BK, 1};
+    if (int e = encode_map(&tk, k, 4, dims, strides, box)) return e;
+    if (int e = encode_map(&tv, v, 4, dims, strides, box)) return e;
+  }
+  DecodeParams p;
+  p.q = reinterpret_cast<const __nv_bfloat16*>(q);
+  p.part = reinterpret_cast<float*>(workspace);
+  p.out = reinterpret_cast<__nv_bfloat16*>(out);
+  p.B = B;
+  p.N = N;
+  p.H_q = H_q;
+  p.H_kv = H_kv;
+  p.splits = sp.splits;
+  p.tiles_per_split = sp.tiles_per_split;
+  p.n_parts = sp.n_parts;
+  p.heads_per_cta = sp.heads_per_cta;
+  p.scale_log2 = (float)((double)scale * 1.4426950408889634);
+  p.status = st->status;
+  p.timeout_ns = g_wait_ns.load();
+  const dim3 grid((unsigned)sp.splits, (unsigned)sp.hblocks, (unsigned)(B * H_kv));
+  sqa::decode_split_kernel<D><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tk, tv, p);
+  if (cudaGetLastError() != cudaSuccess) return SQA_ERR_CUDA;
+  const long long rows = (long long)B * H_q;
+  if (rows > INT_MAX) return SQA_ERR_INVALID_ARG;
+  sqa::decode_combine_kernel<D><<<(unsigned)rows, 128, 0, stream>>>(p);
+  return cudaGetLastError() == cudaSuccess ? SQA_OK : SQA_ERR_CUDA;
+}
+
 template <int D>
 int launch_attn_bwd(const DeviceState* st, const void* q, const void* k, const void* v, const void* out,
                     const void* dout, const float* lse, void* dq, void* dk, void* dv, void* workspace, int B, int N,
@@ -434,6 +502,29 @@ int sqa_attn_bwd(const void* q, const void* k, const void* v, const void* out, c
              ? launch_attn_bwd<64>(st, q, k, v, out, dout, lse, dq, dk, dv, workspace, B, N, H_q, H_kv, causal, scale, s)
              : launch_attn_bwd<128>(st, q, k, v, out, dout, lse, dq, dk, dv, workspace, B, N, H_q, H_kv, causal, scale,
                                     s);
+}
+
+size_t sqa_decode_workspace_bytes(int B, int N, int H_q, int H_kv, int d_head) {
+  if (B < 1 || N < 1 || H_q < 1 || H_kv < 1 || H_kv > H_q || (d_head != 64 && d_head != 128)) return 0;
+  const DecodeSplit sp = decode_split(B, N, H_q, H_kv, d_head);
+  return align256((size_t)B * H_q * sp.n_parts * (d_head + 2) * 4);
+}
+
+int sqa_decode_fwd(const void* q, const void* k_cache, const void* v_cache, void* out, void* workspace,
+                   size_t workspace_bytes, int B, int N, int H_q, int H_kv, int d_head, float scale, void* stream) {
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out)) return SQA_ERR_INVALID_ARG;
+  if (B < 1 || N < 1 || H_q < 1 || H_kv < 1 || H_kv > H_q) return SQA_ERR_INVALID_ARG;
+  if (!(scale > 0.0f) || !std::isfinite(scale)) return SQA_ERR_INVALID_ARG;
+  if (d_head != 64 && d_head != 128) return SQA_ERR_UNSUPPORTED;
+  if ((long double)B * N * H_kv * d_head * 2 >= (long double)(1ull << 40)) return SQA_ERR_INVALID_ARG;
+  const size_t need = sqa_decode_workspace_bytes(B, N, H_q, H_kv, d_head);
+  if (workspace == nullptr || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 || workspace_bytes < need)
+    return SQA_ERR_WORKSPACE;
+  DeviceState* st = nullptr;
+  if (int e = device_state(&st)) return e;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  return d_head == 64 ? launch_decode<64>(st, q, k_cache, v_cache, out, workspace, B, N, H_q, H_kv, scale, s)
+                      : launch_decode<128>(st, q, k_cache, v_cache, out, workspace, B, N, H_q, H_kv, scale, s);
 }
 
 size_t sqa_layer_workspace_bytes(int B, int N, int d_model, int H_q, int H_kv, int d_head) {

@@ -109,3 +109,21 @@ def test_wait_limit_roundtrip(sqa):
     assert sqa.sqa_set_wait_limit_ns(0) == 12345
     assert sqa.sqa_set_wait_limit_ns(prev) == 2_000_000_000
     assert sqa.lib.sqa_check_wait_timeout(10, None) == 1      # limit below range -> invalid
+
+
+def test_decode_workspace_size_and_validation(sqa):
+    assert sqa.sqa_decode_workspace_bytes(0, 128, 8, 2, 64) == 0
+    assert sqa.sqa_decode_workspace_bytes(1, 128, 2, 4, 64) == 0      # H_kv > H_q
+    assert sqa.sqa_decode_workspace_bytes(1, 128, 8, 2, 96) == 0      # unsupported head size
+    small = sqa.sqa_decode_workspace_bytes(1, 128, 8, 2, 64)
+    big = sqa.sqa_decode_workspace_bytes(4, 32768, 16, 4, 128)
+    assert small > 0 and big > small and small % 256 == 0 and big % 256 == 0
+    fake = 1 << 20                                                      # aligned, never dereferenced
+    ws = sqa.sqa_decode_workspace_bytes(1, 128, 8, 2, 64)
+    for args, code in [((None, fake, fake, fake, fake, ws, 1, 128, 8, 2, 64, 0.1), sqa.SQA_ERR_INVALID_ARG),
+                       ((fake, fake, fake, fake, fake, ws, 1, 128, 2, 4, 64, 0.1), sqa.SQA_ERR_INVALID_ARG),
+                       ((fake, fake, fake, fake, fake, ws, 1, 128, 8, 2, 64, -1.0), sqa.SQA_ERR_INVALID_ARG),
+                       ((fake, fake, fake, fake, fake, ws, 1, 128, 8, 2, 80, 0.1), sqa.SQA_ERR_UNSUPPORTED),
+                       ((fake, fake, fake, fake, fake + 8, ws, 1, 128, 8, 2, 64, 0.1), sqa.SQA_ERR_WORKSPACE),
+                       ((fake, fake, fake, fake, fake, ws - 1, 1, 128, 8, 2, 64, 0.1), sqa.SQA_ERR_WORKSPACE)]:
+        assert sqa.sqa_decode_fwd(*args, stream=0, raise_on_error=False) == code, args
