@@ -81,8 +81,10 @@ struct BwdParams {
 
 // Both main kernels run a two-buffer pipeline over 64-column steps. TMEM
 // buffer b (b = step & 1) holds the step's scores in [128b, 128b + 64) and
-// its dP in [128b + 64, 128b + 128); the elementwise warpgroup that owns the
-// buffer writes P / dS back as bf16 over the first 32 columns of each half.
+// its dP in [128b + 64, 128b + 128). Both elementwise warpgroups work on
+// every step, each on its own 32 of the 64 columns, and write P / dS back as
+// bf16 into the first 16 columns of their own 32 (the MMA reads each K16 step
+// of the A operand from wherever its warpgroup put it).
 // Each buffer has its own MMA issuer (warp 1 for even steps, warp 3 for odd
 // steps) with its own gradient accumulators, summed in the epilogue: while one
 // issuer waits for its warpgroup, the other's products keep the tensor core
@@ -91,8 +93,8 @@ struct BwdParams {
 //   warp 0      TMA producer
 //   warp 1      MMA issuer 0 + TMEM owner
 //   warp 3      MMA issuer 1
-//   warps 4-7   elementwise for even steps (thread = TMEM lane = tile row)
-//   warps 8-11  elementwise for odd steps
+//   warps 4-7   elementwise, columns 0-31 of every step (thread = TMEM lane = tile row)
+//   warps 8-11  elementwise, columns 32-63 of every step
 
 // 16 columns of the elementwise step from the scores s and dP read from TMEM:
 // p = exp2(s * scale_log2 - lse2), ds = p * (dP - D), both packed to bf16
@@ -184,7 +186,7 @@ __global__ void __launch_bounds__(384, 1)
 
   WaitCtl ctl{abort_flag, p.status, p.timeout_ns};
   if (tid == 0) {
-    for (int i = 0; i < C::N_BARS; ++i) mbar_init(bar(i), (i == C::BAR_P || i == C::BAR_P + 1) ? 4 : 1);
+    for (int i = 0; i < C::N_BARS; ++i) mbar_init(bar(i), (i == C::BAR_P || i == C::BAR_P + 1) ? 8 : 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -277,8 +279,10 @@ __global__ void __launch_bounds__(384, 1)
           const uint32_t acc = (s > me || kk > 0) ? 1u : 0u;
           const uint64_t ob = (uint64_t)((kk * 16 * 128) >> 4);
           // dV += P^T dO_s and dK += dS^T Q_s (B operands MN-major: d contiguous)
-          umma_ts(col_dv, buf + kk * 8, dDm + so + ob, IDESC_G, acc);
-          umma_ts(col_dk, buf + 64 + kk * 8, dQm + so + ob, IDESC_G, acc);
+          // queries 16kk.. were packed by warpgroup kk/2 into its half, chunk kk%2
+          const uint32_t ca = (uint32_t)(32 * (kk >> 1) + 8 * (kk & 1));
+          umma_ts(col_dv, buf + ca, dDm + so + ob, IDESC_G, acc);
+          umma_ts(col_dk, buf + 64 + ca, dQm + so + ob, IDESC_G, acc);
         }
         umma_commit(bar(C::BAR_EMPTY + st));
         if (s + 2 < n_steps) ok = issue_scores(s + 2);
@@ -290,49 +294,43 @@ __global__ void __launch_bounds__(384, 1)
       mbar_wait(bar(C::BAR_DRAIN + me), 0, drain);
     }
   } else if (warp >= 4) {
-    const int wg = (warp - 4) >> 2;          // 0: even steps, 1: odd steps
+    const int wg = (warp - 4) >> 2;          // 0: columns 0-31 of each step, 1: columns 32-63
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
     const int key = u * 128 + row;
     const uint32_t lane_base = tmem + (uint32_t(quarter * 32) << 16);
-    const uint32_t buf = lane_base + (uint32_t)wg * 128;
+    const int half = 32 * wg;   // this warpgroup's 32 query columns of every step
     const float sl2 = p.scale_log2;
     bool ok = true;
-    for (int s = wg; s < n_steps; s += 2) {
+    for (int s = 0; s < n_steps; ++s) {
       const int st = s % C::STAGES;
       const int t = t_start + s % per_head;
-      // The two warpgroups take turns: step s starts once step s - 1 is done,
-      // so each runs alone while the tensor core works on the other buffer
-      // (run together, they finish together and leave the tensor core idle).
-      if (!mbar_wait_warp(bar(C::BAR_S + wg), (s >> 1) & 1, ctl) ||
-          !mbar_wait_warp(bar(C::BAR_FULL + st), (s / C::STAGES) & 1, ctl) ||
-          (s > 0 && !mbar_wait_warp(bar(C::BAR_P + (wg ^ 1)), ((s - 1) >> 1) & 1, ctl))) {
+      const uint32_t buf = lane_base + (uint32_t)(s & 1) * 128 + (uint32_t)half;
+      if (!mbar_wait_warp(bar(C::BAR_S + (s & 1)), (s >> 1) & 1, ctl) ||
+          !mbar_wait_warp(bar(C::BAR_FULL + st), (s / C::STAGES) & 1, ctl)) {
         ok = false;
         break;
       }
       tc_fence_after();
-      const float4* vl4 = reinterpret_cast<const float4*>(smem + C::OFF_VEC + st * 2 * C::VEC_BYTES);
+      const float4* vl4 = reinterpret_cast<const float4*>(smem + C::OFF_VEC + st * 2 * C::VEC_BYTES) + half / 4;
       const float4* vd4 = vl4 + C::BQ / 4;
       // a key above a query of the step only on the two diagonal tiles; ragged ends
       const bool need_mask = (p.causal && t < 2 * u + 2) || (t * C::BQ + C::BQ > p.N) || (key >= p.N);
-      // four 16-column chunks; chunk k + 1's TMEM load is in flight while
-      // chunk k is computed
+      // two 16-column chunks; chunk 1's TMEM load is in flight while chunk 0 is computed
       uint32_t a0[16], b0[16], a1[16], b1[16];
       tmem_ld16x2_nowait(buf, buf + 64, a0, b0);
       tmem_ld_wait16x2(a0, b0);
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        uint32_t(&ra)[16] = (k & 1) ? a1 : a0;
-        uint32_t(&rb)[16] = (k & 1) ? b1 : b0;
-        uint32_t(&na)[16] = (k & 1) ? a0 : a1;
-        uint32_t(&nb)[16] = (k & 1) ? b0 : b1;
-        if (k < 3) tmem_ld16x2_nowait(buf + 16 * (k + 1), buf + 64 + 16 * (k + 1), na, nb);
+      for (int k = 0; k < 2; ++k) {
+        uint32_t(&ra)[16] = k ? a1 : a0;
+        uint32_t(&rb)[16] = k ? b1 : b0;
+        if (k == 0) tmem_ld16x2_nowait(buf + 16, buf + 64 + 16, a1, b1);
         // masked scores become -inf (p = 0) in a pass of their own, so the
         // arithmetic stays one straight block
         if (need_mask) {
 #pragma unroll
           for (int x = 0; x < 16; ++x) {
-            const int q = t * C::BQ + k * 16 + x;
+            const int q = t * C::BQ + half + k * 16 + x;
             if (q >= p.N || key >= p.N || (p.causal && key > q)) ra[x] = __float_as_uint(-INFINITY);
           }
         }
@@ -347,15 +345,15 @@ __global__ void __launch_bounds__(384, 1)
         }
         uint32_t pp[8], pd[8];
         bwd_chunk(ra, rb, sl2, nl, nd, pp, pd);
-        // chunk k packs into [8k, 8k + 8): behind the columns already read
+        // chunk k packs into [8k, 8k + 8) of this half: behind the columns already read
         tmem_st8(buf + k * 8, pp);
         tmem_st8(buf + 64 + k * 8, pd);
-        if (k < 3) tmem_ld_wait16x2(na, nb);
+        if (k == 0) tmem_ld_wait16x2(a1, b1);
       }
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(bar(C::BAR_P + wg));
+      if (lane == 0) mbar_arrive(bar(C::BAR_P + (s & 1)));
     }
     // epilogue: warpgroup 0 writes dV, warpgroup 1 writes dK (x scale), each
     // the sum over the issuers' accumulators
@@ -469,7 +467,7 @@ __global__ void __launch_bounds__(384, 1)
   WaitCtl ctl{abort_flag, p.status, p.timeout_ns};
   if (tid == 0) {
     for (int i = 0; i < C::N_BARS; ++i)
-      mbar_init(bar(i), (i == C::BAR_P || i == C::BAR_P + 1) ? 4 : ((C::A_TMEM && i == C::BAR_QD) ? 8 : 1));
+      mbar_init(bar(i), (i == C::BAR_P || i == C::BAR_P + 1 || (C::A_TMEM && i == C::BAR_QD)) ? 8 : 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -556,7 +554,7 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
         for (int kk = 0; kk < C::BK / 16; ++kk)
           // dQ += dS K_j (K as an MN-major B operand: d contiguous)
-          umma_ts(col_dq, buf + kk * 8, dKm + so + (uint64_t)((kk * 16 * 128) >> 4), IDESC_G,
+          umma_ts(col_dq, buf + (uint32_t)(32 * (kk >> 1) + 8 * (kk & 1)), dKm + so + (uint64_t)((kk * 16 * 128) >> 4), IDESC_G,
                   (j > me || kk > 0) ? 1u : 0u);
         umma_commit(bar(C::BAR_EMPTY + st));
         if (j + 2 < n_kv) ok = issue_scores(j + 2);
@@ -575,7 +573,7 @@ __global__ void __launch_bounds__(384, 1)
     const int head = head0 + (row & (p.P - 1));
     const bool row_ok = token < p.N;
     const uint32_t lane_base = tmem + (uint32_t(quarter * 32) << 16);
-    const uint32_t buf = lane_base + (uint32_t)wg * 128;
+    const int half = 32 * wg;   // this warpgroup's 32 key columns of every step
     const float sl2 = p.scale_log2;
     float nl_r = 0.f, nd_r = 0.f;
     if (row_ok) {
@@ -606,13 +604,9 @@ __global__ void __launch_bounds__(384, 1)
       nd[w] = make_float2(nd_r, nd_r);
     }
     bool ok = true;
-    for (int j = wg; j < n_kv; j += 2) {
-      // the warpgroups take turns (see the dK/dV kernel)
-      if (!mbar_wait_warp(bar(C::BAR_S + wg), (j >> 1) & 1, ctl) ||
-          (j > 0 && !mbar_wait_warp(bar(C::BAR_P + (wg ^ 1)), ((j - 1) >> 1) & 1, ctl))) {
-        ok = false;
-        break;
-      }
+    for (int j = 0; j < n_kv; ++j) {
+      const uint32_t buf = lane_base + (uint32_t)(j & 1) * 128 + (uint32_t)half;
+      if (!mbar_wait_warp(bar(C::BAR_S + (j & 1)), (j >> 1) & 1, ctl)) { ok = false; break; }
       tc_fence_after();
       // keys above t0 only in the last tiles when causal; keys past N in the last tile
       const bool need_mask = !row_ok || (j * C::BK + C::BK > p.N) || (p.causal && j * C::BK + C::BK - 1 > t0);
@@ -620,28 +614,26 @@ __global__ void __launch_bounds__(384, 1)
       tmem_ld16x2_nowait(buf, buf + 64, a0, b0);
       tmem_ld_wait16x2(a0, b0);
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        uint32_t(&ra)[16] = (k & 1) ? a1 : a0;
-        uint32_t(&rb)[16] = (k & 1) ? b1 : b0;
-        uint32_t(&na)[16] = (k & 1) ? a0 : a1;
-        uint32_t(&nb)[16] = (k & 1) ? b0 : b1;
-        if (k < 3) tmem_ld16x2_nowait(buf + 16 * (k + 1), buf + 64 + 16 * (k + 1), na, nb);
+      for (int k = 0; k < 2; ++k) {
+        uint32_t(&ra)[16] = k ? a1 : a0;
+        uint32_t(&rb)[16] = k ? b1 : b0;
+        if (k == 0) tmem_ld16x2_nowait(buf + 16, buf + 64 + 16, a1, b1);
         if (need_mask) {   // masked scores -> -inf (p = 0), outside the arithmetic block
 #pragma unroll
           for (int x = 0; x < 16; ++x) {
-            const int key = j * C::BK + k * 16 + x;
+            const int key = j * C::BK + half + k * 16 + x;
             if (!row_ok || key >= p.N || (p.causal && key > token)) ra[x] = __float_as_uint(-INFINITY);
           }
         }
         uint32_t pp[8], pd[8];
         bwd_chunk(ra, rb, sl2, nl, nd, pp, pd);
         tmem_st8(buf + k * 8, pd);
-        if (k < 3) tmem_ld_wait16x2(na, nb);
+        if (k == 0) tmem_ld_wait16x2(a1, b1);
       }
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(bar(C::BAR_P + wg));
+      if (lane == 0) mbar_arrive(bar(C::BAR_P + (j & 1)));
     }
     // epilogue: each warpgroup writes half of the row's d columns (x scale),
     // the sum of the two issuers' accumulators
