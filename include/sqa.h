@@ -73,6 +73,24 @@ int sqa_attn_fwd_lse(const void* q, const void* k, const void* v, void* out, flo
                      int causal, float scale, void* stream);
 
 /*
+ * Attention for a contiguous block of query rows: the rows at global
+ * positions q_offset .. q_offset + N_q - 1 of a sequence of N_k tokens,
+ * against all N_k keys (causal: key u visible iff u <= q_offset + t). This is
+ * the per-rank step of sequence sharding, where each rank owns a block of
+ * query positions and gathers every key and value.
+ *   q   [B, N_q, H_q,  d_head]  (the block's query rows)
+ *   k   [B, N_k, H_kv, d_head]
+ *   v   [B, N_k, H_kv, d_head]
+ *   out [B, N_q, H_q,  d_head]  written in full
+ * Requirements as sqa_attn_fwd, plus N_q >= 1, q_offset >= 0 and
+ * q_offset + N_q <= N_k. Results equal rows q_offset .. q_offset + N_q - 1 of
+ * sqa_attn_fwd over the whole sequence.
+ */
+int sqa_attn_fwd_rows(const void* q, const void* k, const void* v, void* out,
+                      int B, int N_q, int N_k, int q_offset, int H_q, int H_kv, int d_head,
+                      int causal, float scale, void* stream);
+
+/*
  * Bytes of device workspace sqa_attn_bwd needs (two fp32 [B, H_q] x N row
  * arrays, rows padded to a multiple of 4 floats). Returns 0 for invalid sizes.
  */

@@ -14,7 +14,7 @@ from .build import LIB as _LIB_PATH
 
 __all__ = [
     "SQA_OK", "SQA_ERR_INVALID_ARG", "SQA_ERR_UNSUPPORTED", "SQA_ERR_CUDA", "SQA_ERR_TIMEOUT",
-    "SQA_ERR_WORKSPACE", "SqaError", "lib", "EXPORTED_SYMBOLS", "sqa_attn_fwd", "sqa_attn_fwd_lse",
+    "SQA_ERR_WORKSPACE", "SqaError", "lib", "EXPORTED_SYMBOLS", "sqa_attn_fwd", "sqa_attn_fwd_lse", "sqa_attn_fwd_rows",
     "sqa_attn_bwd_workspace_bytes", "sqa_attn_bwd", "sqa_decode_workspace_bytes", "sqa_decode_fwd", "sqa_layer_fwd",
     "sqa_layer_workspace_bytes", "sqa_layer_fwd_static_ws", "SQA_STATIC_WORKSPACE_BYTES", "sqa_linear_fwd",
     "sqa_device_status", "sqa_set_wait_limit_ns",
@@ -25,7 +25,7 @@ SQA_OK, SQA_ERR_INVALID_ARG, SQA_ERR_UNSUPPORTED, SQA_ERR_CUDA, SQA_ERR_TIMEOUT,
 SQA_STATIC_WORKSPACE_BYTES = 64 << 20   # include/sqa.h
 
 EXPORTED_SYMBOLS = (
-    "sqa_attn_fwd", "sqa_attn_fwd_lse", "sqa_attn_bwd_workspace_bytes", "sqa_attn_bwd",
+    "sqa_attn_fwd", "sqa_attn_fwd_lse", "sqa_attn_fwd_rows", "sqa_attn_bwd_workspace_bytes", "sqa_attn_bwd",
     "sqa_decode_workspace_bytes", "sqa_decode_fwd", "sqa_layer_workspace_bytes", "sqa_layer_fwd", "sqa_layer_fwd_static_ws", "sqa_linear_fwd",
     "sqa_device_status",
     "sqa_set_wait_limit_ns", "sqa_check_wait_timeout", "sqa_status_string", "sqa_version",
@@ -43,6 +43,8 @@ lib.sqa_attn_fwd.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _vp
 lib.sqa_attn_fwd.restype = _i
 lib.sqa_attn_fwd_lse.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _vp]
 lib.sqa_attn_fwd_lse.restype = _i
+lib.sqa_attn_fwd_rows.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _f, _vp]
+lib.sqa_attn_fwd_rows.restype = _i
 lib.sqa_attn_bwd_workspace_bytes.argtypes = [_i, _i, _i]
 lib.sqa_attn_bwd_workspace_bytes.restype = _sz
 lib.sqa_attn_bwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _i, _i, _i, _i, _i, _i, _f, _vp]
@@ -115,6 +117,14 @@ def sqa_attn_fwd_lse(q, k, v, out, lse, B, N, H_q, H_kv, d_head, causal, scale, 
     st = lib.sqa_attn_fwd_lse(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, N, H_q, H_kv, d_head,
                               int(causal), float(scale), _stream(stream))
     return _check(st, "sqa_attn_fwd_lse", raise_on_error)
+
+
+def sqa_attn_fwd_rows(q, k, v, out, B, N_q, N_k, q_offset, H_q, H_kv, d_head, causal, scale, stream=None,
+                      raise_on_error=True):
+    """Rows q_offset .. q_offset+N_q-1 of attention over N_k tokens (q/out [B,N_q,H_q,d], k/v [B,N_k,H_kv,d])."""
+    st = lib.sqa_attn_fwd_rows(_ptr(q), _ptr(k), _ptr(v), _ptr(out), B, N_q, N_k, q_offset, H_q, H_kv, d_head,
+                               int(causal), float(scale), _stream(stream))
+    return _check(st, "sqa_attn_fwd_rows", raise_on_error)
 
 
 def sqa_attn_bwd_workspace_bytes(B, N, H_q):

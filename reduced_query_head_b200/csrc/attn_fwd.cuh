@@ -36,7 +36,9 @@ namespace sqa {
 
 struct AttnParams {
   __nv_bfloat16* out;   // [B, N, H_q, D]
-  int B, N, H_q, H_kv;
+  int B, N, H_q, H_kv;  // N: query rows of this call
+  int Nk;               // keys (N_k >= q0 + N); N_k = N and q0 = 0 for whole-sequence attention
+  int q0;               // global position of query row 0 (causal masks compare global positions)
   int P, log2P;         // heads stacked per tile
   int tpt;              // tokens per 128-row tile = 128 / P
   int n_pairs;          // tile pairs per (batch, head block)
@@ -137,7 +139,7 @@ __global__ void __launch_bounds__(384, 1)
   const int b = rest / p.n_hb;
   const int head0 = hb * p.P;
   const int g = (int)(((long long)head0 * p.H_kv) / p.H_q);
-  const int n_kv_all = (p.N + C::BN - 1) / C::BN;
+  const int n_kv_all = (p.Nk + C::BN - 1) / C::BN;
   int t0[2], n_kv[2];
 #pragma unroll
   for (int k = 0; k < 2; ++k) {
@@ -146,8 +148,8 @@ __global__ void __launch_bounds__(384, 1)
     if (t0[k] >= p.N) {
       n_kv[k] = 0;
     } else if (p.causal) {
-      const int last = min(t0[k] + p.tpt - 1, p.N - 1);
-      n_kv[k] = last / C::BN + 1;
+      const int last = p.q0 + min(t0[k] + p.tpt - 1, p.N - 1);  // global position of the tile's last row
+      n_kv[k] = min(last / C::BN + 1, n_kv_all);
     } else {
       n_kv[k] = n_kv_all;
     }
@@ -387,7 +389,7 @@ __global__ void __launch_bounds__(384, 1)
     const float sl2 = p.scale_log2;
     const float2 sl2x2 = make_float2(sl2, sl2);
     const int nk = n_kv[k];
-    const int t_first = t0[k];
+    const int t_first = p.q0 + t0[k];   // global position of the tile's first row
     float m = -INFINITY, l = 0.f;
     bool ok = true;
     for (int j = 0; j < nk; ++j) {
@@ -406,10 +408,10 @@ __global__ void __launch_bounds__(384, 1)
       if (lane == 0) mbar_arrive(bar(C::BAR_SFREE + k));
 
       const int key0 = j * C::BN;
-      const bool tail = key0 + C::BN > p.N;
+      const bool tail = key0 + C::BN > p.Nk;
       const bool diag = p.causal && (key0 + C::BN - 1 > t_first);
       if (tail || diag) {
-        const int lim = p.causal ? min(token, p.N - 1) : p.N - 1;  // last visible key
+        const int lim = p.causal ? min(p.q0 + token, p.Nk - 1) : p.Nk - 1;  // last visible key
 #pragma unroll
         for (int u = 0; u < 128; ++u)
           if (key0 + u > lim) s[u] = -INFINITY;

@@ -184,9 +184,13 @@ int heads_per_tile(int H_q, int H_kv) {
 }
 
 template <int D>
+// N query rows at global positions q0 .. q0 + N - 1 against Nk keys (Nk < 0:
+// Nk = N, the whole-sequence case).
 int launch_attn(const DeviceState* st, const void* q, const void* k, const void* v, void* out, int B, int N, int H_q,
-                int H_kv, int causal, float scale, cudaStream_t stream, float* lse = nullptr) {
+                int H_kv, int causal, float scale, cudaStream_t stream, float* lse = nullptr, int Nk = -1,
+                int q0 = 0) {
   using C = AttnCfg<D>;
+  if (Nk < 0) Nk = N;
   const int P = heads_per_tile(H_q, H_kv);
   int log2P = 0;
   while ((1 << log2P) < P) ++log2P;
@@ -213,13 +217,15 @@ int launch_attn(const DeviceState* st, const void* q, const void* k, const void*
     if (int e = encode_map(&tq, q, 4, dims, strides, box)) return e;
   }
   {
-    const cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)H_kv, (cuuint64_t)N, (cuuint64_t)B};
-    const cuuint64_t strides[3] = {(cuuint64_t)D * 2, (cuuint64_t)H_kv * D * 2, (cuuint64_t)N * H_kv * D * 2};
+    const cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)H_kv, (cuuint64_t)Nk, (cuuint64_t)B};
+    const cuuint64_t strides[3] = {(cuuint64_t)D * 2, (cuuint64_t)H_kv * D * 2, (cuuint64_t)Nk * H_kv * D * 2};
     const cuuint32_t box[4] = {64, 1, (cuuint32_t)C::BN, 1};
     if (int e = encode_map(&tk, k, 4, dims, strides, box)) return e;
     if (int e = encode_map(&tv, v, 4, dims, strides, box)) return e;
   }
   AttnParams p;
+  p.Nk = Nk;
+  p.q0 = q0;
   p.out = reinterpret_cast<__nv_bfloat16*>(out);
   p.B = B;
   p.N = N;
@@ -479,6 +485,18 @@ int sqa_attn_fwd_lse(const void* q, const void* k, const void* v, void* out, flo
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   return d_head == 64 ? launch_attn<64>(st, q, k, v, out, B, N, H_q, H_kv, causal, scale, s, lse)
                       : launch_attn<128>(st, q, k, v, out, B, N, H_q, H_kv, causal, scale, s, lse);
+}
+
+int sqa_attn_fwd_rows(const void* q, const void* k, const void* v, void* out, int B, int N_q, int N_k, int q_offset,
+                      int H_q, int H_kv, int d_head, int causal, float scale, void* stream) {
+  if (N_k < 1 || N_q < 1 || q_offset < 0 || (long long)q_offset + N_q > N_k) return SQA_ERR_INVALID_ARG;
+  if (int e = check_attn_args(q, k, v, out, B, N_k, H_q, H_kv, d_head, causal, scale)) return e;
+  DeviceState* st = nullptr;
+  if (int e = device_state(&st)) return e;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  return d_head == 64
+             ? launch_attn<64>(st, q, k, v, out, B, N_q, H_q, H_kv, causal, scale, s, nullptr, N_k, q_offset)
+             : launch_attn<128>(st, q, k, v, out, B, N_q, H_q, H_kv, causal, scale, s, nullptr, N_k, q_offset);
 }
 
 size_t sqa_attn_bwd_workspace_bytes(int B, int N, int H_q) {

@@ -127,3 +127,13 @@ def test_decode_workspace_size_and_validation(sqa):
                        ((fake, fake, fake, fake, fake + 8, ws, 1, 128, 8, 2, 64, 0.1), sqa.SQA_ERR_WORKSPACE),
                        ((fake, fake, fake, fake, fake, ws - 1, 1, 128, 8, 2, 64, 0.1), sqa.SQA_ERR_WORKSPACE)]:
         assert sqa.sqa_decode_fwd(*args, stream=0, raise_on_error=False) == code, args
+
+
+def test_rows_argument_validation(sqa):
+    fake = 1 << 20
+    for n_q, n_k, off, code in [(0, 128, 0, sqa.SQA_ERR_INVALID_ARG), (64, 128, 65, sqa.SQA_ERR_INVALID_ARG),
+                                (64, 128, -1, sqa.SQA_ERR_INVALID_ARG), (1, 0, 0, sqa.SQA_ERR_INVALID_ARG)]:
+        assert sqa.sqa_attn_fwd_rows(fake, fake, fake, fake, 1, n_q, n_k, off, 8, 2, 64, 1, 0.125, stream=0,
+                                     raise_on_error=False) == code
+    assert sqa.sqa_attn_fwd_rows(fake, fake, fake, fake, 1, 64, 128, 0, 8, 2, 96, 1, 0.125, stream=0,
+                                 raise_on_error=False) == sqa.SQA_ERR_UNSUPPORTED
