@@ -273,14 +273,40 @@ def bench_sqa(args):
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
+    # Uploads, kernels and downloads run on three streams so that the copies of
+    # one head configuration overlap the kernels of the others (PCIe is full
+    # duplex): config i+1's q/k/v go up while config i computes, and config i's
+    # output comes down while config i+1 computes. A configuration's device
+    # buffers are rewritten only after its previous kernel has finished.
+    up, down = torch.cuda.Stream(device=device), torch.cuda.Stream(device=device)
+    computed = [torch.cuda.Event() for _ in cfgs]
+    for c_i in range(len(cfgs)):
+        computed[c_i].record(stream)
     for s in range(args.steps):
         flush.fill_((s + 1) & 0xFF)
         e2e_ev[s][0].record(stream)
-        for c in cfgs:
-            for name in ("q", "k", "v"):
-                c["dev"][name].copy_(c["host"][name], non_blocking=True)
+        up.wait_event(e2e_ev[s][0])
+        uploaded, downloaded = [], []
+        for c_i, c in enumerate(cfgs):
+            up.wait_event(computed[c_i])
+            with torch.cuda.stream(up):
+                for name in ("q", "k", "v"):
+                    c["dev"][name].copy_(c["host"][name], non_blocking=True)
+            ev_up = torch.cuda.Event()
+            ev_up.record(up)
+            uploaded.append(ev_up)
+        for c_i, c in enumerate(cfgs):
+            stream.wait_event(uploaded[c_i])
             launch(c)
-            c["out_host"].copy_(c["out"], non_blocking=True)
+            computed[c_i] = torch.cuda.Event()
+            computed[c_i].record(stream)
+            down.wait_event(computed[c_i])
+            with torch.cuda.stream(down):
+                c["out_host"].copy_(c["out"], non_blocking=True)
+            ev_down = torch.cuda.Event()
+            ev_down.record(down)
+            downloaded.append(ev_down)
+        stream.wait_event(downloaded[-1])
         e2e_ev[s][1].record(stream)
     torch.cuda.synchronize()
     e2e_ms = sum(a.elapsed_time(b) for a, b in e2e_ev) / args.steps
