@@ -640,6 +640,38 @@ def _bench_extra(args, sqa, torch, device, stream, flush, peaks, lines):
                           "frac_of_hbm": round(gbs / peaks["hbm_gbs"], 3), "bytes": int(nbytes)})
             print(json.dumps(lines[-1]), flush=True)
             del q, k, v, out, ws
+    elif args.workload == "encoder":
+        # encoder-style (non-causal) layer on one long sequence, the SQA abstract's compute-bound
+        # scenario: x [1, N, 2048], d_head 64, per head configuration
+        import synth
+        B, N, dm, d = 1, args.N, 2048, 64
+
+        def mk(shape, name, factor):
+            h = torch.empty(shape, dtype=torch.bfloat16)
+            synth.fill_bf16_into(h.data_ptr(), h.numel(), 0, name, factor)
+            return h.to(device)
+        x = mk((B, N, dm), "x", 1.0)
+        out = torch.empty((B, N, dm), dtype=torch.bfloat16, device=device)
+        for name, H_q, H_kv in (("MHA", 16, 16), ("GQA", 16, 4), ("SQA", 8, 4), ("xSQA", 4, 4)):
+            wq, wk, wv = mk((H_q * d, dm), "wq", 0.02), mk((H_kv * d, dm), "wk", 0.02), mk((H_kv * d, dm), "wv", 0.02)
+            wo = mk((dm, H_q * d), "wo", 0.02)
+            ws_bytes = sqa.sqa_layer_workspace_bytes(B, N, dm, H_q, H_kv, d)
+            ws = torch.empty(ws_bytes, dtype=torch.uint8, device=device)
+
+            def fn():
+                sqa.sqa_layer_fwd(x, wq, wk, wv, wo, out, ws, ws_bytes, B, N, dm, H_q, H_kv, d, 0, 0.125, stream)
+            for _ in range(args.warmup):
+                fn()
+            ms = _time_launches(fn, args.steps, flush, stream)
+            assert sqa.sqa_device_status(stream) == 0
+            med = statistics.median(ms)
+            fl_attn = attn_flops(B, N, H_q, d, False)
+            fl_gemm = 2.0 * B * N * dm * (H_q + 2 * H_kv) * d + 2.0 * B * N * (H_q * d) * dm
+            lines.append({"workload": "encoder", "config": name, "N": N, "H_q": H_q, "H_kv": H_kv, "d": d,
+                          "d_model": dm, "ms_per_layer": round(med, 3),
+                          "tflops_total": round((fl_attn + fl_gemm) / (med * 1e-3) / 1e12, 1)})
+            print(json.dumps(lines[-1]), flush=True)
+            del wq, wk, wv, wo, ws
     elif args.workload == "layer":
         import synth
         B, N, dm, H_q, H_kv, d = 4, 16384, 2048, 16, 8, 64
@@ -689,7 +721,8 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["sqa", "reference"], default="sqa")
-    ap.add_argument("--workload", choices=["headcfg32k", "small", "long", "layer", "sweep", "single", "linear", "bwd", "decode"],
+    ap.add_argument("--workload", choices=["headcfg32k", "small", "long", "layer", "sweep", "single", "linear", "bwd", "decode",
+                             "encoder"],
                     default="headcfg32k")
     ap.add_argument("--N", type=int, default=32768)
     ap.add_argument("--B", type=int, default=8, help="sequences per decode step (--workload decode)")

@@ -82,3 +82,16 @@ def test_config4_causal_layer_sampled():
     f = [oracle.widen_bf16(b) for b in bits]
     want = oracle.layer_rows(f[0], f[1], f[2], f[3], f[4], rows, H_q, H_kv, d, True, 0.125, storage_rounding=True)
     assert_close(got, want, "config4 layer")
+
+
+def test_encoder_layer_noncausal_sampled():
+    """Encoder-style (non-causal) SQA layer on one long sequence: x [1,32768,2048], H_q=8, H_kv=4."""
+    import torch
+    B, N, dm, H_q, H_kv, d = 1, 32768, 2048, 8, 4, 64
+    bits = _layer_inputs(B, N, dm, H_q, H_kv, d, 5)
+    out = _run_layer(bits, B, N, dm, H_q, H_kv, d, False, 0.125)
+    rows = sampled_rows(B, N, 5)
+    got = bf16_tensor_to_f64(out.view(B * N, dm)[torch.from_numpy(rows).cuda()])
+    f = [oracle.widen_bf16(b) for b in bits]
+    want = oracle.layer_rows(f[0], f[1], f[2], f[3], f[4], rows, H_q, H_kv, d, False, 0.125, storage_rounding=True)
+    assert_close(got, want, "encoder layer")
