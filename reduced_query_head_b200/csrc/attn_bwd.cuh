@@ -85,11 +85,13 @@ struct BwdParams {
 // every step, each on its own 32 of the 64 columns, and write P / dS back as
 // bf16 into the first 16 columns of their own 32 (the MMA reads each K16 step
 // of the A operand from wherever its warpgroup put it).
-// Each buffer has its own MMA issuer (warp 1 for even steps, warp 3 for odd
-// steps) with its own gradient accumulators, summed in the epilogue: while one
-// issuer waits for its warpgroup, the other's products keep the tensor core
-// busy. (The dK/dV kernel at d = 128 has no TMEM left for a second set of
-// accumulators and runs one issuer over both buffers.)
+// dQ kernel: each buffer has its own MMA issuer (warp 1 for even steps, warp 3
+// for odd steps) with its own dQ accumulator, summed in the epilogue: while one
+// issuer waits for the elementwise warps, the other's products keep the tensor
+// core busy. dK/dV kernel at d = 64: K and V sit in TMEM, so all four products
+// are TS; warp 1 issues S^T and dV, warp 3 dP^T and dK, and every TMEM region
+// (scores or dP half of a buffer, one accumulator) has a single issuer. At
+// d = 128 there is no TMEM left for K and V; one issuer runs every product.
 //   warp 0      TMA producer
 //   warp 1      MMA issuer 0 + TMEM owner
 //   warp 3      MMA issuer 1
@@ -119,7 +121,9 @@ template <int D>
 struct DkdvCfg {
   static constexpr int KCH = D / 64;                   // 128-byte column chunks
   static constexpr int BQ = 64;                        // queries per step
-  static constexpr int NI = (D == 64) ? 2 : 1;         // MMA issuers (see above)
+  // d = 64: K and V rows in TMEM (A operands of the score products), two issuers
+  static constexpr bool KV_TMEM = (D == 64);
+  static constexpr int NI = KV_TMEM ? 2 : 1;
   static constexpr int STAGES = (D == 64) ? 8 : 4;
   static constexpr int KV_BYTES = 128 * D * 2;         // K or V tile, 128 keys
   static constexpr int KV_CHUNK = 128 * 128;           // one column chunk of it
@@ -127,7 +131,7 @@ struct DkdvCfg {
   static constexpr int T_CHUNK = BQ * 128;
   static constexpr int STAGE_BYTES = 2 * T_BYTES;
   static constexpr int VEC_BYTES = BQ * 4;             // -lse2 or -D of the step's queries
-  static constexpr int OFF_K = 0, OFF_V = KV_BYTES, OFF_STAGE = 2 * KV_BYTES;
+  static constexpr int OFF_K = 0, OFF_V = KV_BYTES, OFF_STAGE = KV_TMEM ? 0 : 2 * KV_BYTES;
   static constexpr int OFF_VEC = OFF_STAGE + STAGES * STAGE_BYTES;   // [STAGES][-lse2 | -D]
   static constexpr int OFF_BAR = OFF_VEC + STAGES * 2 * VEC_BYTES;
   static constexpr int BAR_KV = 0, BAR_FULL = 1, BAR_EMPTY = 1 + STAGES, BAR_S = 1 + 2 * STAGES,
@@ -136,9 +140,9 @@ struct DkdvCfg {
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
   static constexpr int THREADS = 384;
   static constexpr uint32_t TMEM_COLS = 512;
-  // accumulators of issuer i: dV at COL_ACC + i * ACC_STRIDE, dK D columns after it
-  static constexpr uint32_t COL_ACC = 256, ACC_STRIDE = 2 * D;
-  static_assert(COL_ACC + NI * ACC_STRIDE <= TMEM_COLS, "TMEM budget");
+  // dV at COL_ACC, dK D columns after it; K and V rows (KV_TMEM) after those
+  static constexpr uint32_t COL_ACC = 256, COL_KT = COL_ACC + 2 * D, COL_VT = COL_KT + D / 2;
+  static_assert(COL_ACC + 2 * D <= TMEM_COLS && (!KV_TMEM || COL_VT + D / 2 <= TMEM_COLS), "TMEM budget");
   static_assert(STAGE_BYTES % 1024 == 0 && OFF_STAGE % 1024 == 0, "tile alignment");
 };
 
@@ -186,7 +190,14 @@ __global__ void __launch_bounds__(384, 1)
 
   WaitCtl ctl{abort_flag, p.status, p.timeout_ns};
   if (tid == 0) {
-    for (int i = 0; i < C::N_BARS; ++i) mbar_init(bar(i), (i == C::BAR_P || i == C::BAR_P + 1) ? 8 : 1);
+    // KV_TMEM: the 8 elementwise warps arrive on BAR_KV after writing K / V
+    // into TMEM; S and EMPTY then take one commit from each issuer
+    for (int i = 0; i < C::N_BARS; ++i) {
+      int cnt = 1;
+      if (i == C::BAR_P || i == C::BAR_P + 1 || (C::KV_TMEM && i == C::BAR_KV)) cnt = 8;
+      else if (C::KV_TMEM && ((i >= C::BAR_S && i < C::BAR_S + 2) || (i >= C::BAR_EMPTY && i < C::BAR_EMPTY + C::STAGES))) cnt = 2;
+      mbar_init(bar(i), cnt);
+    }
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -201,11 +212,13 @@ __global__ void __launch_bounds__(384, 1)
 
   if (warp == 0) {
     if (lane == 0) {
-      mbar_arrive_expect_tx(bar(C::BAR_KV), 2 * C::KV_BYTES);
+      if (!C::KV_TMEM) {
+        mbar_arrive_expect_tx(bar(C::BAR_KV), 2 * C::KV_BYTES);
 #pragma unroll
-      for (int c = 0; c < C::KCH; ++c) {
-        tma_load_4d(sbase + C::OFF_K + c * C::KV_CHUNK, &tm_k, bar(C::BAR_KV), c * 64, g, u * 128, b);
-        tma_load_4d(sbase + C::OFF_V + c * C::KV_CHUNK, &tm_v, bar(C::BAR_KV), c * 64, g, u * 128, b);
+        for (int c = 0; c < C::KCH; ++c) {
+          tma_load_4d(sbase + C::OFF_K + c * C::KV_CHUNK, &tm_k, bar(C::BAR_KV), c * 64, g, u * 128, b);
+          tma_load_4d(sbase + C::OFF_V + c * C::KV_CHUNK, &tm_v, bar(C::BAR_KV), c * 64, g, u * 128, b);
+        }
       }
       int filled = 0;
       for (int s = 0; s < n_steps; ++s) {
@@ -227,7 +240,7 @@ __global__ void __launch_bounds__(384, 1)
       }
       volatile int zero = 0;
       WaitCtl drain{&zero, p.status, drain_limit_ns(p.timeout_ns)};
-      mbar_wait(bar(C::BAR_KV), 0, drain);
+      if (!C::KV_TMEM) mbar_wait(bar(C::BAR_KV), 0, drain);
       for (int s = max(0, filled - C::STAGES); s < filled; ++s)
         mbar_wait(bar(C::BAR_FULL + s % C::STAGES), (s / C::STAGES) & 1, drain);
     }
@@ -243,49 +256,82 @@ __global__ void __launch_bounds__(384, 1)
       const uint64_t dDk = sdesc_sw128(sbase + C::OFF_STAGE + C::T_BYTES, 16, 1024);
       const uint64_t dQm = sdesc_sw128(sbase + C::OFF_STAGE, C::T_CHUNK, 1024);
       const uint64_t dDm = sdesc_sw128(sbase + C::OFF_STAGE + C::T_BYTES, C::T_CHUNK, 1024);
-      // S^T = K Q_s^T and dP^T = V dO_s^T into buffer s & 1
-      auto issue_scores = [&](int s) -> bool {
-        const int st = s % C::STAGES;
-        if (!mbar_wait(bar(C::BAR_FULL + st), (s / C::STAGES) & 1, ctl)) return false;
-        tc_fence_after();
-        const uint64_t so = (uint64_t)(st * (C::STAGE_BYTES >> 4));
-        const uint32_t buf = tmem + (uint32_t)(s & 1) * 128;
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint64_t ok_ = ((kk >> 2) * C::KV_CHUNK + (kk & 3) * 32) >> 4;
-          const uint64_t oq = ((kk >> 2) * C::T_CHUNK + (kk & 3) * 32) >> 4;
-          umma_ss(buf, dK + ok_, dQk + so + oq, IDESC_S, kk > 0);
-          umma_ss(buf + 64, dV + ok_, dDk + so + oq, IDESC_S, kk > 0);
-        }
-        umma_commit(bar(C::BAR_S + (s & 1)));
-        return true;
-      };
+      const uint32_t col_dv = tmem + C::COL_ACC, col_dk = col_dv + D;
       bool ok = mbar_wait(bar(C::BAR_KV), 0, ctl);
-      if (C::NI == 2) {
-        if (ok && me < n_steps) ok = issue_scores(me);
+      if (C::KV_TMEM) {
+        // issuer 0: S^T = K Q_s^T into the buffer's first half, dV += P^T dO_s;
+        // issuer 1: dP^T = V dO_s^T into its second half, dK += dS^T Q_s
+        const uint32_t col_a = tmem + (me ? C::COL_VT : C::COL_KT);
+        const uint64_t d_score = me ? dDk : dQk, d_grad = me ? dQm : dDm;
+        const uint32_t col_acc = me ? col_dk : col_dv, half = me ? 64u : 0u;
+        auto issue_score = [&](int s) -> bool {
+          const int st = s % C::STAGES;
+          if (!mbar_wait(bar(C::BAR_FULL + st), (s / C::STAGES) & 1, ctl)) return false;
+          tc_fence_after();
+          const uint64_t so = (uint64_t)(st * (C::STAGE_BYTES >> 4));
+          const uint32_t buf = tmem + (uint32_t)(s & 1) * 128 + half;
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk)
+            umma_ts(buf, col_a + kk * 8, d_score + so + (uint64_t)(((kk & 3) * 32) >> 4), IDESC_S, kk > 0);
+          umma_commit(bar(C::BAR_S + (s & 1)));
+          return true;
+        };
+        if (ok) ok = issue_score(0);
+        if (ok && n_steps > 1) ok = issue_score(1);
+        for (int s = 0; ok && s < n_steps; ++s) {
+          if (!mbar_wait_spin(bar(C::BAR_P + (s & 1)), (s >> 1) & 1, ctl)) { ok = false; break; }
+          tc_fence_after();
+          const int st = s % C::STAGES;
+          const uint64_t so = (uint64_t)(st * (C::STAGE_BYTES >> 4));
+          const uint32_t buf = tmem + (uint32_t)(s & 1) * 128 + half;
+#pragma unroll
+          for (int kk = 0; kk < C::BQ / 16; ++kk)
+            // queries 16kk.. were packed by warpgroup kk/2 into its 32 columns, chunk kk%2
+            umma_ts(col_acc, buf + (uint32_t)(32 * (kk >> 1) + 8 * (kk & 1)), d_grad + so + (uint64_t)((kk * 16 * 128) >> 4),
+                    IDESC_G, (s > 0 || kk > 0) ? 1u : 0u);
+          umma_commit(bar(C::BAR_EMPTY + st));
+          // S^T / dP^T of step s + 2 overwrite what this issuer's own products just read
+          if (s + 2 < n_steps) ok = issue_score(s + 2);
+        }
       } else {
+        // S^T = K Q_s^T and dP^T = V dO_s^T into buffer s & 1
+        auto issue_scores = [&](int s) -> bool {
+          const int st = s % C::STAGES;
+          if (!mbar_wait(bar(C::BAR_FULL + st), (s / C::STAGES) & 1, ctl)) return false;
+          tc_fence_after();
+          const uint64_t so = (uint64_t)(st * (C::STAGE_BYTES >> 4));
+          const uint32_t buf = tmem + (uint32_t)(s & 1) * 128;
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint64_t ok_ = ((kk >> 2) * C::KV_CHUNK + (kk & 3) * 32) >> 4;
+            const uint64_t oq = ((kk >> 2) * C::T_CHUNK + (kk & 3) * 32) >> 4;
+            umma_ss(buf, dK + ok_, dQk + so + oq, IDESC_S, kk > 0);
+            umma_ss(buf + 64, dV + ok_, dDk + so + oq, IDESC_S, kk > 0);
+          }
+          umma_commit(bar(C::BAR_S + (s & 1)));
+          return true;
+        };
         if (ok) ok = issue_scores(0);
         if (ok && n_steps > 1) ok = issue_scores(1);
-      }
-      const uint32_t col_dv = tmem + C::COL_ACC + (uint32_t)me * C::ACC_STRIDE, col_dk = col_dv + D;
-      for (int s = me; ok && s < n_steps; s += C::NI) {
-        if (!mbar_wait_spin(bar(C::BAR_P + (s & 1)), (s >> 1) & 1, ctl)) { ok = false; break; }
-        tc_fence_after();
-        const int st = s % C::STAGES;
-        const uint64_t so = (uint64_t)(st * (C::STAGE_BYTES >> 4));
-        const uint32_t buf = tmem + (uint32_t)(s & 1) * 128;
+        for (int s = 0; ok && s < n_steps; ++s) {
+          if (!mbar_wait_spin(bar(C::BAR_P + (s & 1)), (s >> 1) & 1, ctl)) { ok = false; break; }
+          tc_fence_after();
+          const int st = s % C::STAGES;
+          const uint64_t so = (uint64_t)(st * (C::STAGE_BYTES >> 4));
+          const uint32_t buf = tmem + (uint32_t)(s & 1) * 128;
 #pragma unroll
-        for (int kk = 0; kk < C::BQ / 16; ++kk) {
-          const uint32_t acc = (s > me || kk > 0) ? 1u : 0u;
-          const uint64_t ob = (uint64_t)((kk * 16 * 128) >> 4);
-          // dV += P^T dO_s and dK += dS^T Q_s (B operands MN-major: d contiguous)
-          // queries 16kk.. were packed by warpgroup kk/2 into its half, chunk kk%2
-          const uint32_t ca = (uint32_t)(32 * (kk >> 1) + 8 * (kk & 1));
-          umma_ts(col_dv, buf + ca, dDm + so + ob, IDESC_G, acc);
-          umma_ts(col_dk, buf + 64 + ca, dQm + so + ob, IDESC_G, acc);
+          for (int kk = 0; kk < C::BQ / 16; ++kk) {
+            const uint32_t acc = (s > 0 || kk > 0) ? 1u : 0u;
+            const uint64_t ob = (uint64_t)((kk * 16 * 128) >> 4);
+            // dV += P^T dO_s and dK += dS^T Q_s (B operands MN-major: d contiguous)
+            // queries 16kk.. were packed by warpgroup kk/2 into its half, chunk kk%2
+            const uint32_t ca = (uint32_t)(32 * (kk >> 1) + 8 * (kk & 1));
+            umma_ts(col_dv, buf + ca, dDm + so + ob, IDESC_G, acc);
+            umma_ts(col_dk, buf + 64 + ca, dQm + so + ob, IDESC_G, acc);
+          }
+          umma_commit(bar(C::BAR_EMPTY + st));
+          if (s + 2 < n_steps) ok = issue_scores(s + 2);
         }
-        umma_commit(bar(C::BAR_EMPTY + st));
-        if (s + 2 < n_steps) ok = issue_scores(s + 2);
       }
       if (ok) umma_commit(bar(C::BAR_DONE + me));
       umma_commit(bar(C::BAR_DRAIN + me));
@@ -301,6 +347,23 @@ __global__ void __launch_bounds__(384, 1)
     const uint32_t lane_base = tmem + (uint32_t(quarter * 32) << 16);
     const int half = 32 * wg;   // this warpgroup's 32 query columns of every step
     const float sl2 = p.scale_log2;
+    if constexpr (C::KV_TMEM) {
+      // this key's row of K (warpgroup 0) or V (warpgroup 1) into its TMEM lane; zero past N
+      static_assert(D == 64, "one 32-column TMEM store per row");
+      const __nv_bfloat16* src = (wg == 0 ? p.k : p.v) + (((size_t)b * p.N + (key < p.N ? key : 0)) * p.H_kv + g) * D;
+      const uint4* s4 = reinterpret_cast<const uint4*>(src);
+      uint32_t r[D / 2];
+#pragma unroll
+      for (int x = 0; x < D / 8; ++x) {
+        const uint4 a = key < p.N ? s4[x] : make_uint4(0u, 0u, 0u, 0u);
+        r[4 * x] = a.x; r[4 * x + 1] = a.y; r[4 * x + 2] = a.z; r[4 * x + 3] = a.w;
+      }
+      tmem_st32(lane_base + (wg == 0 ? C::COL_KT : C::COL_VT), r);
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(C::BAR_KV));
+    }
     bool ok = true;
     for (int s = 0; s < n_steps; ++s) {
       const int st = s % C::STAGES;
@@ -355,10 +418,8 @@ __global__ void __launch_bounds__(384, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(C::BAR_P + (s & 1)));
     }
-    // epilogue: warpgroup 0 writes dV, warpgroup 1 writes dK (x scale), each
-    // the sum over the issuers' accumulators
-    const bool two = C::NI == 2 && n_steps > 1;
-    if (ok && mbar_wait_warp(bar(C::BAR_DONE), 0, ctl) && (!two || mbar_wait_warp(bar(C::BAR_DONE + 1), 0, ctl))) {
+    // epilogue: warpgroup 0 writes dV, warpgroup 1 writes dK (x scale)
+    if (ok && mbar_wait_warp(bar(C::BAR_DONE), 0, ctl) && (C::NI == 1 || mbar_wait_warp(bar(C::BAR_DONE + 1), 0, ctl))) {
       tc_fence_after();
       const bool store = key < p.N;
       const size_t base = (((size_t)b * p.N + (store ? key : 0)) * p.H_kv + g) * D;
@@ -367,14 +428,8 @@ __global__ void __launch_bounds__(384, 1)
       const uint32_t col0 = lane_base + C::COL_ACC + (wg == 0 ? 0u : (uint32_t)D);
 #pragma unroll
       for (int c = 0; c < D; c += 32) {
-        uint32_t r[32], r1[32];
-        if (two) {
-          tmem_ld32x2(col0 + c, col0 + C::ACC_STRIDE + c, r, r1);
-#pragma unroll
-          for (int x = 0; x < 32; ++x) r[x] = __float_as_uint(__uint_as_float(r[x]) + __uint_as_float(r1[x]));
-        } else {
-          tmem_ld32(col0 + c, r);
-        }
+        uint32_t r[32];
+        tmem_ld32(col0 + c, r);
         uint4 w[4];
         uint32_t* wp = reinterpret_cast<uint32_t*>(w);
 #pragma unroll
