@@ -278,6 +278,14 @@ def bench_sqa(args):
     # duplex): config i+1's q/k/v go up while config i computes, and config i's
     # output comes down while config i+1 computes. A configuration's device
     # buffers are rewritten only after its previous kernel has finished.
+    # The pipeline's fill is the first configuration's upload and its drain the
+    # last one's download, so the step starts with the smallest upload and ends
+    # with the smallest download (the same work in any order).
+    up_bytes = [sum(t.numel() * 2 for t in c["host"].values()) for c in cfgs]
+    first = min(range(len(cfgs)), key=lambda i: up_bytes[i])
+    rest = [i for i in range(len(cfgs)) if i != first]
+    last = min(rest, key=lambda i: cfgs[i]["out"].numel()) if rest else None
+    order = [first] + [i for i in rest if i != last] + ([last] if last is not None else [])
     up, down = torch.cuda.Stream(device=device), torch.cuda.Stream(device=device)
     computed = [torch.cuda.Event() for _ in cfgs]
     for c_i in range(len(cfgs)):
@@ -286,16 +294,18 @@ def bench_sqa(args):
         flush.fill_((s + 1) & 0xFF)
         e2e_ev[s][0].record(stream)
         up.wait_event(e2e_ev[s][0])
-        uploaded, downloaded = [], []
-        for c_i, c in enumerate(cfgs):
+        uploaded, downloaded = {}, []
+        for c_i in order:
+            c = cfgs[c_i]
             up.wait_event(computed[c_i])
             with torch.cuda.stream(up):
                 for name in ("q", "k", "v"):
                     c["dev"][name].copy_(c["host"][name], non_blocking=True)
             ev_up = torch.cuda.Event()
             ev_up.record(up)
-            uploaded.append(ev_up)
-        for c_i, c in enumerate(cfgs):
+            uploaded[c_i] = ev_up
+        for c_i in order:
+            c = cfgs[c_i]
             stream.wait_event(uploaded[c_i])
             launch(c)
             computed[c_i] = torch.cuda.Event()
@@ -397,12 +407,17 @@ def oracle_sample(rows_per_cfg, seed=0):
 
 
 def cpu_baseline(seconds=15.0):
-    # size the sample from a probe taken after a warm-up call (thread pool,
-    # first-touch allocation), so the whole leg takes about `seconds`
+    # size the sample after a warm-up call (thread pool, first-touch
+    # allocation); the cost per row falls as the sample grows, so rescale until
+    # one sample takes at least 60% of `seconds`
     oracle_sample(8)
-    f1, s1 = oracle_sample(64)
-    rows = int(max(64, min(8192, 64 * seconds / max(s1, 1e-3))))
+    rows = 256
     f, s = oracle_sample(rows)
+    for _ in range(2):
+        if s >= 0.6 * seconds or rows >= 16384:
+            break
+        rows = int(max(rows, min(16384, rows * seconds / max(s, 1e-3))))
+        f, s = oracle_sample(rows)
     return {"value": round(f / s / 1e12, 6), "unit": "TFLOP/s", "cores": _blas_threads(), "kind": "oracle",
             "sample": "%d query positions (all heads) of each of the 7 head configs at N=32768, d=64, "
                       "float64 numpy/BLAS; %.1f s" % (rows, s)}
