@@ -452,11 +452,17 @@ def bench_reference(args):
 
 
 # ---------------------------------------------------------------------- extra workloads
-def _time_launches(fn, reps, flush, stream):
+def _time_launches(fn, reps, flush, stream, evict=None):
+    """CUDA-event time of each of `reps` calls of fn, the L2 flushed before each by a write of
+    `flush`. With `evict`, a read of that second buffer (also larger than L2) follows the write,
+    so the dirty lines of the flush are written back before the timed region instead of inside
+    it (that write-back is a sizeable part of a kernel lasting tens of microseconds)."""
     import torch
     evs = []
     for r in range(reps):
         flush.fill_(r & 0xFF)
+        if evict is not None:
+            evict.sum(dtype=torch.int64)
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
         fn()
@@ -472,19 +478,20 @@ def bench_extra(args):
     device = torch.device("cuda", 0)
     stream = torch.cuda.current_stream()
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+    evict = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)   # see _time_launches
     peaks = load_peaks()
     lines = []
     clocks = ClockSampler(0)
     clocks.start()
     try:
-        _bench_extra(args, sqa, torch, device, stream, flush, peaks, lines)
+        _bench_extra(args, sqa, torch, device, stream, flush, evict, peaks, lines)
     finally:
         clk = clocks.stop()
     print(json.dumps({"workload": args.workload, "clocks": clk}), flush=True)
     return lines
 
 
-def _bench_extra(args, sqa, torch, device, stream, flush, peaks, lines):
+def _bench_extra(args, sqa, torch, device, stream, flush, evict, peaks, lines):
     if args.workload in ("long", "sweep"):
         if args.workload == "long":
             grid = [(N, H_q, H_kv, 64, c, 1.0, 0) for N in (65536, 131072, 200000)
@@ -527,7 +534,7 @@ def _bench_extra(args, sqa, torch, device, stream, flush, peaks, lines):
             sqa.sqa_attn_fwd(dev["q"], dev["k"], dev["v"], out, B, N, H_q, H_kv, d, 0, 0.125, stream)
         for _ in range(max(args.warmup, 3)):
             fn()
-        cold = _time_launches(fn, args.steps, flush, stream)
+        cold = _time_launches(fn, args.steps, flush, stream, evict)
         warm_ev = []
         for _ in range(args.steps):
             a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -645,7 +652,7 @@ def _bench_extra(args, sqa, torch, device, stream, flush, peaks, lines):
                 sqa.sqa_decode_fwd(q, k, v, out, ws, ws_bytes, B, N, H_q, H_kv, d, d ** -0.5, stream)
             for _ in range(args.warmup):
                 fn()
-            ms = _time_launches(fn, args.steps, flush, stream)
+            ms = _time_launches(fn, args.steps, flush, stream, evict)
             assert sqa.sqa_device_status(stream) == 0
             med = statistics.median(ms)
             nbytes = 2.0 * B * N * H_kv * d * 2 + 2.0 * 2 * B * H_q * d

@@ -19,7 +19,9 @@
 //                         measured slower: barriers and atomics per CTA.)
 //   decode_combine_kernel merges the partials of each (b, i) into out (one
 //                         CTA per head row; each thread reads a 16-column
-//                         slice of a strided set of parts).
+//                         slice of a strided set of parts). It is launched as
+//                         a programmatic dependent of the split grid, so its
+//                         launch overlaps the split's last wave.
 #pragma once
 
 #include "sm100.cuh"
@@ -273,6 +275,10 @@ __global__ void __launch_bounds__(160)
       }
     }
   }
+  // the combine grid (launched as a programmatic dependent) may be scheduled
+  // once every CTA of this grid got here or exited; its griddepcontrol.wait
+  // still waits for this grid to complete and its writes to be visible
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
 // One CTA of 128 threads per (b, i): merge the partials of all splits and
@@ -287,6 +293,9 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(const DecodeParams 
   __shared__ float gl[G];
   const int row = blockIdx.x;   // b * H_q + i
   const int t = threadIdx.x;
+  // launched as a programmatic dependent of the split grid: wait until that
+  // grid has completed and its partials are visible (a no-op otherwise)
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const float* base = p.part + (size_t)row * p.n_parts * (D + 2);
   // the largest partial maximum (parts that saw no key hold -inf)
   float M = -INFINITY;

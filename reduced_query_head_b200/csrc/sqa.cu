@@ -4,6 +4,7 @@
 #include <cuda_runtime.h>
 
 #include <atomic>
+#include <algorithm>
 #include <climits>
 #include <cmath>
 #include <cstdint>
@@ -309,24 +310,37 @@ int bwd_row_ld(int N) { return (N + 3) & ~3; }
 size_t bwd_vec_bytes(int B, int N, int H_q) { return align256((size_t)B * H_q * bwd_row_ld(N) * 4); }
 
 // Decode work split: the keys of each (b, g, head block) are cut into `splits`
-// ranges of whole 64-key tiles, aiming at about four waves of the two resident
-// CTAs on each of 148 SMs (many short CTAs balance the SMs; each still streams
-// several tiles). A pure function of the sizes, so the workspace size is too.
+// ranges of whole 64-key tiles. The split count minimises a small cost model:
+// waves of the 296 resident CTAs (two per SM on 148 SMs) times the tiles one
+// CTA streams plus about three tiles' worth of pipeline fill. Few long CTAs
+// when the cache is small (one wave), enough CTAs to fill whole waves when it
+// is large. A pure function of the sizes, so the workspace size is too.
 struct DecodeSplit {
   int hblocks, splits, tiles_per_split, n_parts, heads_per_cta;
 };
 DecodeSplit decode_split(int B, int N, int H_q, int H_kv, int d) {
+  constexpr long long kResident = 2 * 148;   // decode_split_kernel CTAs resident at once
+  constexpr long long kFillTiles = 3;        // pipeline fill of one CTA, in tiles
   DecodeSplit r;
   r.heads_per_cta = 16 * (d == 64 ? DecodeCfg<64>::RB : DecodeCfg<128>::RB);
   const int r_max = (H_q + H_kv - 1) / H_kv;
   r.hblocks = (r_max + r.heads_per_cta - 1) / r.heads_per_cta;
-  const int n_tiles = (N + 63) / 64;
+  const long long n_tiles = (N + 63) / 64;
   const long long base = (long long)B * H_kv * r.hblocks;
-  long long want = (4 * 296 + base - 1) / base;
-  if (want < 1) want = 1;
-  if (want > n_tiles) want = n_tiles;
-  r.tiles_per_split = (int)((n_tiles + want - 1) / want);
-  r.splits = (n_tiles + r.tiles_per_split - 1) / r.tiles_per_split;
+  // more splits than eight waves' worth only add partials
+  const long long s_max = std::max(1LL, std::min(n_tiles, (8 * kResident + base - 1) / base));
+  long long best_tps = n_tiles, best_cost = -1;
+  for (long long sp = 1; sp <= s_max; ++sp) {
+    const long long tps = (n_tiles + sp - 1) / sp;
+    const long long ctas = base * ((n_tiles + tps - 1) / tps);
+    const long long cost = ((ctas + kResident - 1) / kResident) * (tps + kFillTiles);
+    if (best_cost < 0 || cost < best_cost) {
+      best_cost = cost;
+      best_tps = tps;
+    }
+  }
+  r.tiles_per_split = (int)best_tps;
+  r.splits = (int)((n_tiles + best_tps - 1) / best_tps);
   r.n_parts = 4 * r.splits;
   return r;
 }
@@ -365,7 +379,19 @@ int launch_decode(const DeviceState* st, const void* q, const void* k, const voi
   if (cudaGetLastError() != cudaSuccess) return SQA_ERR_CUDA;
   const long long rows = (long long)B * H_q;
   if (rows > INT_MAX) return SQA_ERR_INVALID_ARG;
-  sqa::decode_combine_kernel<D><<<(unsigned)rows, 128, 0, stream>>>(p);
+  // programmatic dependent launch: the combine's launch overlaps the split's
+  // tail; the kernel's griddepcontrol.wait orders it after the split grid
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)rows);
+  cfg.blockDim = dim3(128);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, sqa::decode_combine_kernel<D>, p) != cudaSuccess) return SQA_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? SQA_OK : SQA_ERR_CUDA;
 }
 
