@@ -280,12 +280,15 @@ def bench_sqa(args):
     # buffers are rewritten only after its previous kernel has finished.
     # The pipeline's fill is the first configuration's upload and its drain the
     # last one's download, so the step starts with the smallest upload and ends
-    # with the smallest download (the same work in any order).
+    # with the smallest download. In between, configurations go in increasing
+    # order of upload bytes per FLOP, so the upload stream stays ahead of the
+    # kernels (the same work in any order).
     up_bytes = [sum(t.numel() * 2 for t in c["host"].values()) for c in cfgs]
     first = min(range(len(cfgs)), key=lambda i: up_bytes[i])
     rest = [i for i in range(len(cfgs)) if i != first]
     last = min(rest, key=lambda i: cfgs[i]["out"].numel()) if rest else None
-    order = [first] + [i for i in rest if i != last] + ([last] if last is not None else [])
+    middle = sorted((i for i in rest if i != last), key=lambda i: up_bytes[i] / cfgs[i]["flops"])
+    order = [first] + middle + ([last] if last is not None else [])
     up, down = torch.cuda.Stream(device=device), torch.cuda.Stream(device=device)
     computed = [torch.cuda.Event() for _ in cfgs]
     for c_i in range(len(cfgs)):
