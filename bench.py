@@ -278,17 +278,8 @@ def bench_sqa(args):
     # duplex): config i+1's q/k/v go up while config i computes, and config i's
     # output comes down while config i+1 computes. A configuration's device
     # buffers are rewritten only after its previous kernel has finished.
-    # The pipeline's fill is the first configuration's upload and its drain the
-    # last one's download, so the step starts with the smallest upload and ends
-    # with the smallest download. In between, configurations go in increasing
-    # order of upload bytes per FLOP, so the upload stream stays ahead of the
-    # kernels (the same work in any order).
-    up_bytes = [sum(t.numel() * 2 for t in c["host"].values()) for c in cfgs]
-    first = min(range(len(cfgs)), key=lambda i: up_bytes[i])
-    rest = [i for i in range(len(cfgs)) if i != first]
-    last = min(rest, key=lambda i: cfgs[i]["out"].numel()) if rest else None
-    middle = sorted((i for i in rest if i != last), key=lambda i: up_bytes[i] / cfgs[i]["flops"])
-    order = [first] + middle + ([last] if last is not None else [])
+    order = pipeline_order([sum(t.numel() * 2 for t in c["host"].values()) for c in cfgs],
+                           [c["out"].numel() * 2 for c in cfgs], [c["flops"] for c in cfgs])
     up, down = torch.cuda.Stream(device=device), torch.cuda.Stream(device=device)
     computed = [torch.cuda.Event() for _ in cfgs]
     for c_i in range(len(cfgs)):
@@ -407,6 +398,27 @@ def oracle_sample(rows_per_cfg, seed=0):
         secs += time.perf_counter() - t0
         flops += 4.0 * len(rows) * N * H_q * d
     return flops, secs
+
+
+def pipeline_order(up_bytes, down_bytes, flops):
+    """Order of the head configurations in one end-to-end step.
+
+    The pipeline's fill is the first configuration's upload and its drain the
+    last one's download, so the step starts with the smallest upload and ends
+    with the smallest download of the rest. In between, configurations go in
+    increasing order of upload bytes per FLOP, so the upload stream stays ahead
+    of the kernels. The work is the same in any order.
+    """
+    n = len(up_bytes)
+    if n == 0:
+        return []
+    first = min(range(n), key=lambda i: up_bytes[i])
+    rest = [i for i in range(n) if i != first]
+    if not rest:
+        return [first]
+    last = min(rest, key=lambda i: down_bytes[i])
+    middle = sorted((i for i in rest if i != last), key=lambda i: up_bytes[i] / flops[i])
+    return [first] + middle + [last]
 
 
 def cpu_baseline(seconds=15.0):
