@@ -147,6 +147,11 @@ size_t sqa_decode_workspace_bytes(int B, int N, int H_q, int H_kv, int d_head);
  * Requirements: B, N >= 1; 1 <= H_kv <= H_q; d_head in {64, 128}; scale
  * finite and > 0. Arithmetic: bf16 inputs, fp32 scores, softmax and sums, P
  * rounded to bf16 for the P.V product, bf16 output.
+ * Errors: SQA_ERR_INVALID_ARG for bad pointers, sizes or scale;
+ * SQA_ERR_UNSUPPORTED for other head sizes; SQA_ERR_WORKSPACE for a null,
+ * misaligned or short workspace. Enqueues two kernels on `stream`: the split
+ * pass and the merge, the merge as a programmatic dependent launch of the
+ * split (it starts early and waits on the device for the split to finish).
  */
 int sqa_decode_fwd(const void* q, const void* k_cache, const void* v_cache, void* out,
                    void* workspace, size_t workspace_bytes,
