@@ -456,7 +456,11 @@ __global__ void __launch_bounds__(384, 1)
 template <int D>
 struct DqCfg {
   static constexpr int KCH = D / 64;
-  static constexpr int BK = 64;                        // keys per step
+  // d = 64 (SPLIT): issuer 0 issues S, issuer 1 issues dP and dQ, so one dQ
+  // accumulator suffices and the TMEM it frees holds 96-key steps; d = 128:
+  // one issuer per buffer, each with its own dQ accumulator, 64-key steps.
+  static constexpr bool SPLIT = (D == 64);
+  static constexpr int BK = SPLIT ? 96 : 64;           // keys per step
   static constexpr int STAGES = (D == 64) ? 8 : 4;
   // d = 64: Q and dO live in TMEM as the A operands of the score products (TS
   // form); at d = 128 the two issuers' accumulators fill TMEM and they stay in
@@ -475,16 +479,28 @@ struct DqCfg {
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
   static constexpr int THREADS = 384;
   static constexpr uint32_t TMEM_COLS = 512;
-  // dQ accumulator of issuer i at COL_DQ + i * D; Q / dO rows (A_TMEM) after them
-  static constexpr uint32_t COL_DQ = 256, COL_QT = 256 + 2 * D, COL_DOT = COL_QT + D / 2;
-  static_assert(COL_DQ + 2 * D <= TMEM_COLS && (!A_TMEM || COL_DOT + D / 2 <= TMEM_COLS), "TMEM budget");
+  // TMEM buffer b at b * BUF: scores in [0, BK), dP in [BK, 2 BK). Then the dQ
+  // accumulator(s) (issuer i's at COL_DQ + i * D when not SPLIT), then the Q /
+  // dO rows (A_TMEM).
+  static constexpr uint32_t BUF = 2 * BK, N_ACC = SPLIT ? 1 : 2;
+  static constexpr uint32_t COL_DQ = 2 * BUF, COL_QT = COL_DQ + N_ACC * D, COL_DOT = COL_QT + D / 2;
+  static_assert(COL_DQ + N_ACC * D <= TMEM_COLS && (!A_TMEM || COL_DOT + D / 2 <= TMEM_COLS), "TMEM budget");
+  static_assert(!SPLIT || A_TMEM, "the split issuers take Q and dO from TMEM");
+  // elementwise: each warpgroup owns CPW key columns of a step, in NCH chunks
+  // of 16; chunk k of warpgroup w packs its dS into [w*CPW + 8k, +8) of the
+  // buffer's dP half, behind the columns it has already read
+  static constexpr int CPW = BK / 2, NCH = CPW / 16;
+  static_assert(CPW % 16 == 0, "chunking");
+  __host__ __device__ static constexpr uint32_t ds_col(int kk) {
+    return (uint32_t)((16 * kk / CPW) * CPW + 8 * ((16 * kk % CPW) / 16));
+  }
   static_assert(STAGE_BYTES % 1024 == 0 && OFF_STAGE % 1024 == 0, "tile alignment");
 };
 
 // One CTA per 128-row query tile: P heads of one group stacked as in the
 // forward (row r = token_local * P + head offset), so each K/V tile serves all
-// P heads. Steps walk 64-key tiles: S = Q K_j^T, dP = dO V_j^T, then
-// dQ += dS K_j with dS read from TMEM.
+// P heads. Steps walk BK-key tiles (96 at d = 64, 64 at d = 128):
+// S = Q K_j^T, dP = dO V_j^T, then dQ += dS K_j with dS read from TMEM.
 template <int D>
 __global__ void __launch_bounds__(384, 1)
     bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
@@ -521,8 +537,14 @@ __global__ void __launch_bounds__(384, 1)
 
   WaitCtl ctl{abort_flag, p.status, p.timeout_ns};
   if (tid == 0) {
-    for (int i = 0; i < C::N_BARS; ++i)
-      mbar_init(bar(i), (i == C::BAR_P || i == C::BAR_P + 1 || (C::A_TMEM && i == C::BAR_QD)) ? 8 : 1);
+    // SPLIT: S and EMPTY take one commit from each issuer
+    for (int i = 0; i < C::N_BARS; ++i) {
+      int cnt = 1;
+      if (i == C::BAR_P || i == C::BAR_P + 1 || (C::A_TMEM && i == C::BAR_QD)) cnt = 8;
+      else if (C::SPLIT && ((i >= C::BAR_S && i < C::BAR_S + 2) || (i >= C::BAR_EMPTY && i < C::BAR_EMPTY + C::STAGES)))
+        cnt = 2;
+      mbar_init(bar(i), cnt);
+    }
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -575,44 +597,90 @@ __global__ void __launch_bounds__(384, 1)
       const uint64_t dKk = sdesc_sw128(sbase + C::OFF_STAGE, 16, 1024);
       const uint64_t dVk = sdesc_sw128(sbase + C::OFF_STAGE + C::T_BYTES, 16, 1024);
       const uint64_t dKm = sdesc_sw128(sbase + C::OFF_STAGE, C::T_CHUNK, 1024);
-      // S = Q K_j^T and dP = dO V_j^T into buffer j & 1
-      auto issue_scores = [&](int j) -> bool {
-        const int st = j % C::STAGES;
-        if (!mbar_wait(bar(C::BAR_FULL + st), (j / C::STAGES) & 1, ctl)) return false;
-        tc_fence_after();
-        const uint64_t so = (uint64_t)(st * (C::STAGE_BYTES >> 4));
-        const uint32_t buf = tmem + (uint32_t)(j & 1) * 128;
+      bool ok = mbar_wait(bar(C::BAR_QD), 0, ctl);
+      if constexpr (C::SPLIT) {
+        // issuer 0: S_j = Q K_j^T into the buffer's first half; issuer 1:
+        // dP_j = dO V_j^T into its second half, then dQ += dS_j K_j with dS_j
+        // read from that half. Each half has one issuing thread, so in-order
+        // issue puts dP(j + 2) after the dQ(j) that read the same columns.
+        auto issue_score = [&](int j) -> bool {
+          const int st = j % C::STAGES;
+          if (!mbar_wait(bar(C::BAR_FULL + st), (j / C::STAGES) & 1, ctl)) return false;
+          tc_fence_after();
+          const uint64_t so = (uint64_t)(st * (C::STAGE_BYTES >> 4));
+          const uint32_t dst = tmem + (uint32_t)(j & 1) * C::BUF + (me ? (uint32_t)C::BK : 0u);
+          const uint32_t a_col = tmem + (me ? C::COL_DOT : C::COL_QT);
+          const uint64_t b_desc = me ? dVk : dKk;
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint64_t ok_ = ((kk >> 2) * C::T_CHUNK + (kk & 3) * 32) >> 4;
-          if (C::A_TMEM) {
-            umma_ts(buf, tmem + C::COL_QT + kk * 8, dKk + so + ok_, IDESC_S, kk > 0);
-            umma_ts(buf + 64, tmem + C::COL_DOT + kk * 8, dVk + so + ok_, IDESC_S, kk > 0);
-          } else {
-            const uint64_t oq = ((kk >> 2) * C::Q_CHUNK + (kk & 3) * 32) >> 4;
-            umma_ss(buf, dQ + oq, dKk + so + ok_, IDESC_S, kk > 0);
-            umma_ss(buf + 64, dO + oq, dVk + so + ok_, IDESC_S, kk > 0);
+          for (int kk = 0; kk < D / 16; ++kk)
+            umma_ts(dst, a_col + kk * 8, b_desc + so + (uint64_t)(((kk & 3) * 32) >> 4), IDESC_S, kk > 0);
+          umma_commit(bar(C::BAR_S + (j & 1)));
+          return true;
+        };
+        if (me == 0) {
+          for (int j = 0; ok && j < n_kv; ++j) {
+            // buffer j & 1 is free once the elementwise warps have read S(j - 2)
+            if (j >= 2 && !mbar_wait_spin(bar(C::BAR_P + (j & 1)), ((j - 2) >> 1) & 1, ctl)) { ok = false; break; }
+            if (!issue_score(j)) { ok = false; break; }
+            umma_commit(bar(C::BAR_EMPTY + j % C::STAGES));
+          }
+        } else {
+          if (ok && n_kv > 0) ok = issue_score(0);
+          if (ok && n_kv > 1) ok = issue_score(1);
+          for (int j = 0; ok && j < n_kv; ++j) {
+            if (!mbar_wait_spin(bar(C::BAR_P + (j & 1)), (j >> 1) & 1, ctl)) { ok = false; break; }
+            tc_fence_after();
+            const int st = j % C::STAGES;
+            const uint64_t so = (uint64_t)(st * (C::STAGE_BYTES >> 4));
+            const uint32_t ds = tmem + (uint32_t)(j & 1) * C::BUF + (uint32_t)C::BK;
+#pragma unroll
+            for (int kk = 0; kk < C::BK / 16; ++kk)
+              // dQ += dS K_j (K as an MN-major B operand: d contiguous)
+              umma_ts(tmem + C::COL_DQ, ds + C::ds_col(kk), dKm + so + (uint64_t)((kk * 16 * 128) >> 4), IDESC_G,
+                      (j > 0 || kk > 0) ? 1u : 0u);
+            umma_commit(bar(C::BAR_EMPTY + st));
+            if (j + 2 < n_kv) ok = issue_score(j + 2);
           }
         }
-        umma_commit(bar(C::BAR_S + (j & 1)));
-        return true;
-      };
-      bool ok = mbar_wait(bar(C::BAR_QD), 0, ctl);
-      if (ok && me < n_kv) ok = issue_scores(me);
-      const uint32_t col_dq = tmem + C::COL_DQ + (uint32_t)me * D;
-      for (int j = me; ok && j < n_kv; j += 2) {
-        if (!mbar_wait_spin(bar(C::BAR_P + (j & 1)), (j >> 1) & 1, ctl)) { ok = false; break; }
-        tc_fence_after();
-        const int st = j % C::STAGES;
-        const uint64_t so = (uint64_t)(st * (C::STAGE_BYTES >> 4));
-        const uint32_t buf = tmem + (uint32_t)(j & 1) * 128;
+      } else {
+        // S = Q K_j^T and dP = dO V_j^T into buffer j & 1
+        auto issue_scores = [&](int j) -> bool {
+          const int st = j % C::STAGES;
+          if (!mbar_wait(bar(C::BAR_FULL + st), (j / C::STAGES) & 1, ctl)) return false;
+          tc_fence_after();
+          const uint64_t so = (uint64_t)(st * (C::STAGE_BYTES >> 4));
+          const uint32_t buf = tmem + (uint32_t)(j & 1) * 128;
 #pragma unroll
-        for (int kk = 0; kk < C::BK / 16; ++kk)
-          // dQ += dS K_j (K as an MN-major B operand: d contiguous)
-          umma_ts(col_dq, buf + (uint32_t)(32 * (kk >> 1) + 8 * (kk & 1)), dKm + so + (uint64_t)((kk * 16 * 128) >> 4), IDESC_G,
-                  (j > me || kk > 0) ? 1u : 0u);
-        umma_commit(bar(C::BAR_EMPTY + st));
-        if (j + 2 < n_kv) ok = issue_scores(j + 2);
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint64_t ok_ = ((kk >> 2) * C::T_CHUNK + (kk & 3) * 32) >> 4;
+            if (C::A_TMEM) {
+              umma_ts(buf, tmem + C::COL_QT + kk * 8, dKk + so + ok_, IDESC_S, kk > 0);
+              umma_ts(buf + 64, tmem + C::COL_DOT + kk * 8, dVk + so + ok_, IDESC_S, kk > 0);
+            } else {
+              const uint64_t oq = ((kk >> 2) * C::Q_CHUNK + (kk & 3) * 32) >> 4;
+              umma_ss(buf, dQ + oq, dKk + so + ok_, IDESC_S, kk > 0);
+              umma_ss(buf + 64, dO + oq, dVk + so + ok_, IDESC_S, kk > 0);
+            }
+          }
+          umma_commit(bar(C::BAR_S + (j & 1)));
+          return true;
+        };
+        if (ok && me < n_kv) ok = issue_scores(me);
+        const uint32_t col_dq = tmem + C::COL_DQ + (uint32_t)me * D;
+        for (int j = me; ok && j < n_kv; j += 2) {
+          if (!mbar_wait_spin(bar(C::BAR_P + (j & 1)), (j >> 1) & 1, ctl)) { ok = false; break; }
+          tc_fence_after();
+          const int st = j % C::STAGES;
+          const uint64_t so = (uint64_t)(st * (C::STAGE_BYTES >> 4));
+          const uint32_t buf = tmem + (uint32_t)(j & 1) * 128;
+#pragma unroll
+          for (int kk = 0; kk < C::BK / 16; ++kk)
+            // dQ += dS K_j (K as an MN-major B operand: d contiguous)
+            umma_ts(col_dq, buf + (uint32_t)(32 * (kk >> 1) + 8 * (kk & 1)), dKm + so + (uint64_t)((kk * 16 * 128) >> 4), IDESC_G,
+                    (j > me || kk > 0) ? 1u : 0u);
+          umma_commit(bar(C::BAR_EMPTY + st));
+          if (j + 2 < n_kv) ok = issue_scores(j + 2);
+        }
       }
       if (ok) umma_commit(bar(C::BAR_DONE + me));
       umma_commit(bar(C::BAR_DRAIN + me));
@@ -628,7 +696,7 @@ __global__ void __launch_bounds__(384, 1)
     const int head = head0 + (row & (p.P - 1));
     const bool row_ok = token < p.N;
     const uint32_t lane_base = tmem + (uint32_t(quarter * 32) << 16);
-    const int half = 32 * wg;   // this warpgroup's 32 key columns of every step
+    const int half = C::CPW * wg;   // this warpgroup's first key column of every step
     const float sl2 = p.scale_log2;
     float nl_r = 0.f, nd_r = 0.f;
     if (row_ok) {
@@ -660,19 +728,22 @@ __global__ void __launch_bounds__(384, 1)
     }
     bool ok = true;
     for (int j = 0; j < n_kv; ++j) {
-      const uint32_t buf = lane_base + (uint32_t)(j & 1) * 128 + (uint32_t)half;
+      // this warpgroup's score columns of buffer j & 1, and its dP columns
+      const uint32_t buf = lane_base + (uint32_t)(j & 1) * C::BUF + (uint32_t)half;
+      const uint32_t dpb = buf + (uint32_t)C::BK;
       if (!mbar_wait_warp(bar(C::BAR_S + (j & 1)), (j >> 1) & 1, ctl)) { ok = false; break; }
       tc_fence_after();
       // keys above t0 only in the last tiles when causal; keys past N in the last tile
       const bool need_mask = !row_ok || (j * C::BK + C::BK > p.N) || (p.causal && j * C::BK + C::BK - 1 > t0);
-      uint32_t a0[16], b0[16], a1[16], b1[16];
-      tmem_ld16x2_nowait(buf, buf + 64, a0, b0);
-      tmem_ld_wait16x2(a0, b0);
+      // NCH 16-column chunks; chunk k + 1's TMEM load is in flight while chunk k is computed
+      uint32_t ra2[2][16], rb2[2][16];
+      tmem_ld16x2_nowait(buf, dpb, ra2[0], rb2[0]);
+      tmem_ld_wait16x2(ra2[0], rb2[0]);
 #pragma unroll
-      for (int k = 0; k < 2; ++k) {
-        uint32_t(&ra)[16] = k ? a1 : a0;
-        uint32_t(&rb)[16] = k ? b1 : b0;
-        if (k == 0) tmem_ld16x2_nowait(buf + 16, buf + 64 + 16, a1, b1);
+      for (int k = 0; k < C::NCH; ++k) {
+        uint32_t(&ra)[16] = ra2[k & 1];
+        uint32_t(&rb)[16] = rb2[k & 1];
+        if (k + 1 < C::NCH) tmem_ld16x2_nowait(buf + 16 * (k + 1), dpb + 16 * (k + 1), ra2[(k + 1) & 1], rb2[(k + 1) & 1]);
         if (need_mask) {   // masked scores -> -inf (p = 0), outside the arithmetic block
 #pragma unroll
           for (int x = 0; x < 16; ++x) {
@@ -682,18 +753,23 @@ __global__ void __launch_bounds__(384, 1)
         }
         uint32_t pp[8], pd[8];
         bwd_chunk(ra, rb, sl2, nl, nd, pp, pd);
-        tmem_st8(buf + k * 8, pd);
-        if (k == 0) tmem_ld_wait16x2(a1, b1);
+        // dS of chunk k into [8k, 8k + 8) of this warpgroup's dP columns (already read)
+        tmem_st8((C::SPLIT ? dpb : buf) + k * 8, pd);
+        if (k + 1 < C::NCH) tmem_ld_wait16x2(ra2[(k + 1) & 1], rb2[(k + 1) & 1]);
       }
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(C::BAR_P + (j & 1)));
     }
-    // epilogue: each warpgroup writes half of the row's d columns (x scale),
-    // the sum of the two issuers' accumulators
-    const bool two = n_kv > 1;
-    if (ok && mbar_wait_warp(bar(C::BAR_DONE), 0, ctl) && (!two || mbar_wait_warp(bar(C::BAR_DONE + 1), 0, ctl))) {
+    // epilogue: each warpgroup writes half of the row's d columns (x scale):
+    // the single accumulator of issuer 1 (SPLIT), else the sum of the two
+    // issuers' accumulators
+    const bool two = !C::SPLIT && n_kv > 1;
+    const bool acc_ready = ok && (C::SPLIT ? mbar_wait_warp(bar(C::BAR_DONE + 1), 0, ctl)
+                                           : (mbar_wait_warp(bar(C::BAR_DONE), 0, ctl) &&
+                                              (!two || mbar_wait_warp(bar(C::BAR_DONE + 1), 0, ctl))));
+    if (acc_ready) {
       tc_fence_after();
       __nv_bfloat16* dst = p.dq + (((size_t)b * p.N + (row_ok ? token : 0)) * p.H_q + head) * D;
 #pragma unroll
