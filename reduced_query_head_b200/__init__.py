@@ -33,7 +33,8 @@ EXPORTED_SYMBOLS = (
 
 if not os.path.exists(_LIB_PATH):
     raise ImportError(
-        "libsqa.so is not built (expected at %s); run `python -m reduced_query_head_b200.build`" % _LIB_PATH)
+        "libsqa.so is not built (expected at %s); run `python reduced_query_head_b200/build.py` "
+        "or `python __graft_entry__.py`" % _LIB_PATH)
 
 lib = ctypes.CDLL(_LIB_PATH)
 
