@@ -354,7 +354,7 @@ def bench_sqa(args):
                          "algorithmic_bytes_per_launch": alg_bytes},
             "e2e": {"value": round(e2e_value, 2), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms_max, 4)},
-            "gpu_launches": args.steps * len(cfgs),
+            "gpu_launches": args.steps * len(cfgs) * world,   # attention launches, all ranks
             "clocks": clk,
             "per_config": per,
             "speedup_vs_flop_ratio": {"t16/t8": round(t16 / t8, 3), "flop_ratio_16/8": 2.0,
