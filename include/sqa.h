@@ -27,6 +27,11 @@
  *   - The library allocates no device memory per call; the layer takes a
  *     caller-provided workspace.
  *   - Thread-safe; each call may target any device (the current one is used).
+ *   - Per device, the first call looks up and keeps device addresses (the
+ *     status word, the static scratch array) and kernel attributes. They
+ *     belong to that device's primary context: do not call the library again
+ *     after cudaDeviceReset() or another teardown of that context in the same
+ *     process.
  */
 #ifndef SQA_H
 #define SQA_H
@@ -245,6 +250,18 @@ unsigned long long sqa_set_wait_limit_ns(unsigned long long ns);
  * clears it. Shows that a stuck wait ends with a status instead of a hang.
  */
 int sqa_check_wait_timeout(unsigned long long limit_ns, void* stream);
+
+/*
+ * Diagnostic: the exp2 the attention kernels evaluate on the FMA pipe for part
+ * of the softmax (the rest uses the hardware ex2 unit), next to CUDA's exp2f.
+ * For i in [0, n): poly[i] = that polynomial 2^x[i], ref[i] = exp2f(x[i]).
+ * The polynomial: x clamped at -125, x = n + f with n = round(x) and
+ * f in [-1/2, 1/2], 2^f from a degree-3 polynomial with minimum maximum
+ * relative error on [-1/2, 1/2] (7.5e-5), 2^n added into the exponent field.
+ * x, poly, ref: DEVICE fp32 arrays, 4-byte aligned; 1 <= n <= 2^31.
+ * SQA_ERR_INVALID_ARG otherwise. Asynchronous on `stream`.
+ */
+int sqa_check_exp2_poly(const float* x, float* poly, float* ref, long long n, void* stream);
 
 /* Human-readable name of a status code (static string). */
 const char* sqa_status_string(int status);

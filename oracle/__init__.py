@@ -37,6 +37,7 @@ import numpy as np
 __all__ = [
     "group_of_head", "repeat_kv", "widen_bf16", "bf16_round", "attention",
     "attention_rows", "linear", "layer", "layer_rows", "attention_lse", "attention_backward",
+    "attention_backward_q_rows", "attention_backward_kv_rows", "attention_backward_bound", "decode",
 ]
 
 
@@ -335,6 +336,82 @@ def attention_backward_q_rows(q_rows, k, v, dout_rows, rows, N: int, causal: boo
 
     _map_pairs(one_head, [(int(b), i) for b in np.unique(bs) for i in range(H_q)])
     return (out, bound) if with_bound else out
+
+
+def attention_backward_kv_rows(q, k, v, dout, kv_rows, causal: bool, scale: float, chunk: int = 128,
+                               with_bound: bool = False):
+    """(dk, dv) for selected key positions only: each [len(kv_rows), H_kv, d].
+
+    ``kv_rows`` are flat positions b*N + u; q, k, v and dout are the full
+    arrays. A key's gradient collects the column u of every query head's
+    softmax, and P[t, u] needs all of score row t (its maximum and sum), as
+    does the row's D = sum_u P[t,u] dP[t,u]. So for each query head i of group
+    g every score row is formed in full, a chunk of query rows at a time,
+    following the steps of :func:`_head_backward` (softmax, dP, the Jacobian's
+    row sum); only the selected key columns are carried on into
+    dV_g[u] += P[:,u]^T dO_i and dK_g[u] += scale * dS[:,u]^T Q_i, summed over
+    the heads of the group. With ``with_bound`` also returns the error scales
+    (ek, ev) of :func:`attention_backward_bound` at those positions.
+    """
+    q, k, v, dout = (np.asarray(t, dtype=np.float64) for t in (q, k, v, dout))
+    kv_rows = np.asarray(kv_rows, dtype=np.int64)
+    B, N, H_q, d = q.shape
+    H_kv = k.shape[2]
+    bs, us = kv_rows // N, kv_rows % N
+    pairs = [(int(b), i) for b in np.unique(bs) for i in range(H_q)]
+    parts = {}
+
+    def one_head(b, i):
+        sel = np.nonzero(bs == b)[0]
+        u_sel = us[sel]
+        g = group_of_head(i, H_q, H_kv)
+        kh = np.array(k[b, :, g, :])      # explicit repetition: head i's own copy
+        vh = np.array(v[b, :, g, :])
+        qh, doh = q[b, :, i, :], dout[b, :, i, :]
+        dk_h = np.zeros((len(sel), d))
+        dv_h = np.zeros((len(sel), d))
+        ek_h = np.zeros((len(sel), d)) if with_bound else None
+        ev_h = np.zeros((len(sel), d)) if with_bound else None
+        keys = np.arange(N)
+        for a in range(0, N, chunk):
+            t_idx = keys[a:a + chunk]
+            n = min(N, int(t_idx[-1]) + 1) if causal else N
+            live = u_sel < n                # keys past the chunk's last row have P = 0 there
+            if not np.any(live):
+                continue
+            s = scale * (qh[t_idx] @ kh[:n].T)     # full score rows of the chunk
+            if causal:
+                s[keys[None, :n] > t_idx[:, None]] = -np.inf
+            m = np.max(s, axis=1, keepdims=True)
+            e = np.exp(s - m)
+            p = e / np.sum(e, axis=1, keepdims=True)
+            dp = doh[t_idx] @ vh[:n].T
+            dsum = np.sum(p * dp, axis=1, keepdims=True)
+            cols = u_sel[live]
+            p_c = p[:, cols]
+            ds_c = p_c * (dp[:, cols] - dsum)
+            dv_h[live] += p_c.T @ doh[t_idx]
+            dk_h[live] += scale * (ds_c.T @ qh[t_idx])
+            if with_bound:
+                arow = np.sum(np.abs(doh[t_idx]) * (p @ np.abs(vh[:n])), axis=1, keepdims=True)
+                eds = _U * np.abs(ds_c) + 2 * _U * p_c * arow
+                ek_h[live] += scale * (eds.T @ np.abs(qh[t_idx]))
+                ev_h[live] += _U * (p_c.T @ np.abs(doh[t_idx]))
+        parts[(b, i)] = (sel, g, dk_h, dv_h, ek_h, ev_h)
+
+    _map_pairs(one_head, pairs)
+    dk = np.zeros((len(kv_rows), H_kv, d))
+    dv = np.zeros_like(dk)
+    ek = np.zeros_like(dk) if with_bound else None
+    ev = np.zeros_like(dk) if with_bound else None
+    for b, i in pairs:                      # a shared group collects every head's gradient
+        sel, g, dk_h, dv_h, ek_h, ev_h = parts[(b, i)]
+        dk[sel, g] += dk_h
+        dv[sel, g] += dv_h
+        if with_bound:
+            ek[sel, g] += ek_h
+            ev[sel, g] += ev_h
+    return (dk, dv, ek, ev) if with_bound else (dk, dv)
 
 
 # ---------------------------------------------------------------------------

@@ -18,7 +18,7 @@ __all__ = [
     "sqa_attn_bwd_workspace_bytes", "sqa_attn_bwd", "sqa_decode_workspace_bytes", "sqa_decode_fwd", "sqa_layer_fwd",
     "sqa_layer_workspace_bytes", "sqa_layer_fwd_static_ws", "SQA_STATIC_WORKSPACE_BYTES", "sqa_linear_fwd",
     "sqa_device_status", "sqa_set_wait_limit_ns",
-    "sqa_check_wait_timeout", "sqa_status_string", "sqa_version",
+    "sqa_check_wait_timeout", "sqa_check_exp2_poly", "sqa_status_string", "sqa_version",
 ]
 
 SQA_OK, SQA_ERR_INVALID_ARG, SQA_ERR_UNSUPPORTED, SQA_ERR_CUDA, SQA_ERR_TIMEOUT, SQA_ERR_WORKSPACE = range(6)
@@ -28,7 +28,7 @@ EXPORTED_SYMBOLS = (
     "sqa_attn_fwd", "sqa_attn_fwd_lse", "sqa_attn_fwd_rows", "sqa_attn_bwd_workspace_bytes", "sqa_attn_bwd",
     "sqa_decode_workspace_bytes", "sqa_decode_fwd", "sqa_layer_workspace_bytes", "sqa_layer_fwd", "sqa_layer_fwd_static_ws", "sqa_linear_fwd",
     "sqa_device_status",
-    "sqa_set_wait_limit_ns", "sqa_check_wait_timeout", "sqa_status_string", "sqa_version",
+    "sqa_set_wait_limit_ns", "sqa_check_wait_timeout", "sqa_check_exp2_poly", "sqa_status_string", "sqa_version",
 )
 
 if not os.path.exists(_LIB_PATH):
@@ -68,6 +68,8 @@ lib.sqa_set_wait_limit_ns.argtypes = [_ull]
 lib.sqa_set_wait_limit_ns.restype = _ull
 lib.sqa_check_wait_timeout.argtypes = [_ull, _vp]
 lib.sqa_check_wait_timeout.restype = _i
+lib.sqa_check_exp2_poly.argtypes = [_vp, _vp, _vp, _ll, _vp]
+lib.sqa_check_exp2_poly.restype = _i
 lib.sqa_status_string.argtypes = [_i]
 lib.sqa_status_string.restype = ctypes.c_char_p
 lib.sqa_version.argtypes = []
@@ -189,6 +191,12 @@ def sqa_set_wait_limit_ns(ns: int) -> int:
 
 def sqa_check_wait_timeout(limit_ns: int, stream=None) -> int:
     return int(lib.sqa_check_wait_timeout(int(limit_ns), _stream(stream)))
+
+
+def sqa_check_exp2_poly(x, poly, ref, n, stream=None, raise_on_error=True):
+    """poly[i] = the kernels' FMA-pipe polynomial 2^x[i], ref[i] = CUDA exp2f(x[i]) (fp32 device arrays)."""
+    st = lib.sqa_check_exp2_poly(_ptr(x), _ptr(poly), _ptr(ref), int(n), _stream(stream))
+    return _check(st, "sqa_check_exp2_poly", raise_on_error)
 
 
 def sqa_status_string(status: int) -> str:

@@ -45,35 +45,14 @@ struct DeviceState {
   int sms = 0;
 };
 
-// Attention kernels by the share of exp2 evaluated on the FMA pipe (eighths
-// of the column pairs; the rest use the MUFU unit).
+// Attention kernels, one per head size. The template's second argument is the
+// share of exp2 evaluated by the FMA-pipe polynomial (eighths of the column
+// pairs; the rest use the MUFU unit): all-MUFU at d = 64, where the softmax
+// bounds the step, and two eighths at d = 128, where it balances the tensor work.
 using AttnKernel = void (*)(const CUtensorMap, const CUtensorMap, const CUtensorMap, const AttnParams);
-constexpr int kEmuChoices[] = {0, 1, 2, 3, 4, 5};
-constexpr int kNumEmu = 6;
-AttnKernel attn_kernel_64(int i) {
-  static const AttnKernel t[kNumEmu] = {sqa::attn_fwd_kernel<64, 0>, sqa::attn_fwd_kernel<64, 1>,
-                                        sqa::attn_fwd_kernel<64, 2>, sqa::attn_fwd_kernel<64, 3>,
-                                        sqa::attn_fwd_kernel<64, 4>, sqa::attn_fwd_kernel<64, 5>};
-  return t[i];
-}
-AttnKernel attn_kernel_128(int i) {
-  static const AttnKernel t[kNumEmu] = {sqa::attn_fwd_kernel<128, 0>, sqa::attn_fwd_kernel<128, 1>,
-                                        sqa::attn_fwd_kernel<128, 2>, sqa::attn_fwd_kernel<128, 3>,
-                                        sqa::attn_fwd_kernel<128, 4>, sqa::attn_fwd_kernel<128, 5>};
-  return t[i];
-}
-// Default split per head size; SQA_EXP2_POLY_EIGHTHS=<0..5> overrides it.
-constexpr int kDefaultEmu64 = 0, kDefaultEmu128 = 2;
-int emu_index(int d) {
-  int want = d == 64 ? kDefaultEmu64 : kDefaultEmu128;
-  if (const char* e = getenv("SQA_EXP2_POLY_EIGHTHS")) {
-    const int v = atoi(e);
-    for (int i = 0; i < kNumEmu; ++i)
-      if (kEmuChoices[i] == v) want = v;
-  }
-  for (int i = 0; i < kNumEmu; ++i)
-    if (kEmuChoices[i] == want) return i;
-  return 0;
+constexpr int kEmu64 = 0, kEmu128 = 2;
+AttnKernel attn_kernel(int d) {
+  return d == 64 ? sqa::attn_fwd_kernel<64, kEmu64> : sqa::attn_fwd_kernel<128, kEmu128>;
 }
 
 std::mutex g_mu;
@@ -99,17 +78,17 @@ int device_state(DeviceState** out) {
     }
     if (cudaGetSymbolAddress(reinterpret_cast<void**>(&st.status), g_sqa_status) != cudaSuccess) return SQA_ERR_CUDA;
     if (cudaDeviceGetAttribute(&st.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return SQA_ERR_CUDA;
-    for (int e = 0; e < kNumEmu; ++e) {
-      if (cudaFuncSetAttribute(attn_kernel_64(e), cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               AttnCfg<64>::SMEM_BYTES) != cudaSuccess ||
-          cudaFuncSetAttribute(attn_kernel_128(e), cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               AttnCfg<128>::SMEM_BYTES) != cudaSuccess)
-        return SQA_ERR_CUDA;
+    if (cudaFuncSetAttribute(attn_kernel(64), cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             AttnCfg<64>::SMEM_BYTES) != cudaSuccess ||
+        cudaFuncSetAttribute(attn_kernel(128), cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             AttnCfg<128>::SMEM_BYTES) != cudaSuccess)
+      return SQA_ERR_CUDA;
+    {
       // The kernels re-split their registers between warpgroups at run time;
       // the split is only valid for the per-thread count they were built for.
       cudaFuncAttributes a64, a128;
-      if (cudaFuncGetAttributes(&a64, attn_kernel_64(e)) != cudaSuccess ||
-          cudaFuncGetAttributes(&a128, attn_kernel_128(e)) != cudaSuccess)
+      if (cudaFuncGetAttributes(&a64, attn_kernel(64)) != cudaSuccess ||
+          cudaFuncGetAttributes(&a128, attn_kernel(128)) != cudaSuccess)
         return SQA_ERR_CUDA;
       if (a64.numRegs != AttnCfg<64>::REGS_LAUNCH || a128.numRegs != AttnCfg<128>::REGS_LAUNCH)
         return SQA_ERR_UNSUPPORTED;
@@ -243,7 +222,7 @@ int launch_attn(const DeviceState* st, const void* q, const void* k, const void*
   p.status = st->status;
   p.timeout_ns = g_wait_ns.load();
   p.lse = lse;
-  const AttnKernel kern = D == 64 ? attn_kernel_64(emu_index(D)) : attn_kernel_128(emu_index(D));
+  const AttnKernel kern = attn_kernel(D);
   kern<<<(unsigned)grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);
   return cudaGetLastError() == cudaSuccess ? SQA_OK : SQA_ERR_CUDA;
 }
@@ -488,6 +467,49 @@ __global__ void wait_probe_kernel(int* status, unsigned long long ns) {
   sqa::mbar_wait_warp(sqa::smem_u32(&barrier), 0, c);  // nothing arrives: must give up
 }
 
+// Evaluates the attention kernels' FMA-pipe exp2 (sqa::exp2_poly2, on pairs)
+// beside CUDA's exp2f, for checking the polynomial against the library routine.
+__global__ void exp2_poly_probe_kernel(const float* x, float* poly, float* ref, long long n) {
+  const long long stride = 2LL * gridDim.x * blockDim.x;
+  for (long long i = 2LL * (blockIdx.x * (long long)blockDim.x + threadIdx.x); i < n; i += stride) {
+    const bool pair = i + 1 < n;
+    const float a = x[i], b = pair ? x[i + 1] : a;
+    const float2 p = sqa::exp2_poly2(make_float2(a, b));
+    poly[i] = p.x;
+    ref[i] = exp2f(a);
+    if (pair) {
+      poly[i + 1] = p.y;
+      ref[i + 1] = exp2f(b);
+    }
+  }
+}
+
+// Layer sizes whose every tensor, workspace region and tensor-map stride stays
+// below 2^40 bytes, and whose projection widths fit the kernels' int fields.
+bool layer_sizes_fit(int B, int N, int d_model, int H_q, int H_kv, int d_head) {
+  const long double M = (long double)B * N;
+  const long double lim = (long double)(1ull << 40);
+  if (M > INT_MAX) return false;
+  if ((long double)H_q * d_head + 2.0L * H_kv * d_head > INT_MAX) return false;
+  if (M * d_model * 2 >= lim || M * (2.0L * H_q + 2.0L * H_kv) * d_head * 2 >= lim) return false;
+  if ((long double)d_model * H_q * d_head * 2 >= lim) return false;
+  return true;
+}
+
+// Every argument check of the layer entry points, before anything else.
+int check_layer_args(const void* x, const void* Wq, const void* Wk, const void* Wv, const void* Wo, const void* out,
+                     int B, int N, int d_model, int H_q, int H_kv, int d_head, int causal, float scale) {
+  if (!aligned16(x) || !aligned16(Wq) || !aligned16(Wk) || !aligned16(Wv) || !aligned16(Wo) || !aligned16(out))
+    return SQA_ERR_INVALID_ARG;
+  if (d_model < 8 || d_model % 8 != 0) return SQA_ERR_INVALID_ARG;
+  if (B < 1 || N < 1 || H_q < 1 || H_kv < 1 || H_kv > H_q) return SQA_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return SQA_ERR_INVALID_ARG;
+  if (!(scale > 0.0f) || !std::isfinite(scale)) return SQA_ERR_INVALID_ARG;
+  if (d_head != 64 && d_head != 128) return SQA_ERR_UNSUPPORTED;
+  if (!layer_sizes_fit(B, N, d_model, H_q, H_kv, d_head)) return SQA_ERR_INVALID_ARG;
+  return SQA_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -573,6 +595,7 @@ int sqa_decode_fwd(const void* q, const void* k_cache, const void* v_cache, void
 
 size_t sqa_layer_workspace_bytes(int B, int N, int d_model, int H_q, int H_kv, int d_head) {
   if (B < 1 || N < 1 || d_model < 8 || H_q < 1 || H_kv < 1 || H_kv > H_q || d_head < 1) return 0;
+  if (!layer_sizes_fit(B, N, d_model, H_q, H_kv, d_head)) return 0;
   const size_t M = (size_t)B * N;
   return align256(M * H_q * d_head * 2) * 2 + align256(M * H_kv * d_head * 2) * 2;
 }
@@ -580,15 +603,8 @@ size_t sqa_layer_workspace_bytes(int B, int N, int d_model, int H_q, int H_kv, i
 int sqa_layer_fwd(const void* x, const void* Wq, const void* Wk, const void* Wv, const void* Wo, void* out,
                   void* workspace, size_t workspace_bytes, int B, int N, int d_model, int H_q, int H_kv, int d_head,
                   int causal, float scale, void* stream) {
-  if (!aligned16(x) || !aligned16(Wq) || !aligned16(Wk) || !aligned16(Wv) || !aligned16(Wo) || !aligned16(out))
-    return SQA_ERR_INVALID_ARG;
-  if (d_model < 8 || d_model % 8 != 0) return SQA_ERR_INVALID_ARG;
-  if (B < 1 || N < 1 || H_q < 1 || H_kv < 1 || H_kv > H_q) return SQA_ERR_INVALID_ARG;
-  if (causal != 0 && causal != 1) return SQA_ERR_INVALID_ARG;
-  if (!(scale > 0.0f) || !std::isfinite(scale)) return SQA_ERR_INVALID_ARG;
-  if (d_head != 64 && d_head != 128) return SQA_ERR_UNSUPPORTED;
+  if (int e = check_layer_args(x, Wq, Wk, Wv, Wo, out, B, N, d_model, H_q, H_kv, d_head, causal, scale)) return e;
   const long long M = (long long)B * N;
-  if (M > INT_MAX || (long double)M * d_model * 2 >= (long double)(1ull << 40)) return SQA_ERR_INVALID_ARG;
   const size_t need = sqa_layer_workspace_bytes(B, N, d_model, H_q, H_kv, d_head);
   if (workspace == nullptr || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 || workspace_bytes < need)
     return SQA_ERR_WORKSPACE;
@@ -669,6 +685,7 @@ int static_workspace(void** out) {
 int sqa_layer_fwd_static_ws(const void* x, const void* Wq, const void* Wk, const void* Wv, const void* Wo, void* out,
                             int B, int N, int d_model, int H_q, int H_kv, int d_head, int causal, float scale,
                             void* stream) {
+  if (int e = check_layer_args(x, Wq, Wk, Wv, Wo, out, B, N, d_model, H_q, H_kv, d_head, causal, scale)) return e;
   const size_t need = sqa_layer_workspace_bytes(B, N, d_model, H_q, H_kv, d_head);
   if (need == 0) return SQA_ERR_INVALID_ARG;
   if (need > (size_t)SQA_STATIC_WORKSPACE_BYTES) return SQA_ERR_WORKSPACE;  // problem too large for the array
@@ -724,6 +741,18 @@ int sqa_check_wait_timeout(unsigned long long limit_ns, void* stream) {
   wait_probe_kernel<<<1, 32, 0, s>>>(st->status, limit_ns);
   if (cudaGetLastError() != cudaSuccess) return SQA_ERR_CUDA;
   return sqa_device_status(stream);
+}
+
+int sqa_check_exp2_poly(const float* x, float* poly, float* ref, long long n, void* stream) {
+  if (x == nullptr || poly == nullptr || ref == nullptr || n < 1 || n > (1LL << 31)) return SQA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(poly) | reinterpret_cast<uintptr_t>(ref)) & 3u)
+    return SQA_ERR_INVALID_ARG;
+  DeviceState* st = nullptr;
+  if (int e = device_state(&st)) return e;
+  const long long pairs = (n + 1) / 2;
+  const long long blocks = std::min<long long>((pairs + 255) / 256, 8LL * st->sms);
+  exp2_poly_probe_kernel<<<(unsigned)blocks, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(x, poly, ref, n);
+  return cudaGetLastError() == cudaSuccess ? SQA_OK : SQA_ERR_CUDA;
 }
 
 const char* sqa_status_string(int status) {

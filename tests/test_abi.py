@@ -137,3 +137,29 @@ def test_rows_argument_validation(sqa):
                                      raise_on_error=False) == code
     assert sqa.sqa_attn_fwd_rows(fake, fake, fake, fake, 1, 64, 128, 0, 8, 2, 96, 1, 0.125, stream=0,
                                  raise_on_error=False) == sqa.SQA_ERR_UNSUPPORTED
+
+
+def test_layer_argument_errors_come_before_the_workspace_check(sqa):
+    # a problem too large for the library's own array, with an argument sqa_layer_fwd rejects:
+    # the argument error is what comes back (nothing touches the device on either path)
+    B, N, dm, H_q, H_kv, d = 4, 16384, 2048, 16, 8, 64
+    f = sqa.lib.sqa_layer_fwd_static_ws
+    ok = (P, P, P, P, P, P)
+    assert f(*ok, B, N, dm, H_q, H_kv, d, 1, ctypes.c_float(0.125), None) == sqa.SQA_ERR_WORKSPACE
+    assert f(*ok, B, N, dm, H_q, H_kv, d, 2, ctypes.c_float(0.125), None) == sqa.SQA_ERR_INVALID_ARG
+    assert f(*ok, B, N, dm, H_q, H_kv, d, 1, ctypes.c_float(0.0), None) == sqa.SQA_ERR_INVALID_ARG
+    assert f(*ok, B, N, dm + 4, H_q, H_kv, d, 1, ctypes.c_float(0.125), None) == sqa.SQA_ERR_INVALID_ARG
+    assert f(P + 8, P, P, P, P, P, B, N, dm, H_q, H_kv, d, 1, ctypes.c_float(0.125), None) == sqa.SQA_ERR_INVALID_ARG
+    assert f(*ok, B, N, dm, H_q, H_kv, 96, 1, ctypes.c_float(0.125), None) == sqa.SQA_ERR_UNSUPPORTED
+
+
+def test_layer_sizes_that_overflow_are_refused(sqa):
+    # head counts whose projection widths or workspace regions do not fit are refused, and the
+    # workspace size query returns 0 for them instead of a wrapped-around small number
+    big = 1 << 26
+    assert sqa.sqa_layer_workspace_bytes(1, 16, 64, big, big, 64) == 0
+    assert sqa.sqa_layer_workspace_bytes(1 << 20, 1 << 10, 64, 1024, 1, 64) == 0
+    st = sqa.lib.sqa_layer_fwd(P, P, P, P, P, P, P, 1 << 40, 1, 16, 64, big, big, 64, 0, ctypes.c_float(0.125), None)
+    assert st == sqa.SQA_ERR_INVALID_ARG
+    st = sqa.lib.sqa_layer_fwd_static_ws(P, P, P, P, P, P, 1, 16, 64, big, big, 64, 0, ctypes.c_float(0.125), None)
+    assert st == sqa.SQA_ERR_INVALID_ARG

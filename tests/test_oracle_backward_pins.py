@@ -237,3 +237,55 @@ def test_q_rows_bound_matches_full_bound():
     _, b = oracle.attention_backward_q_rows(q[0][rows], k, v, dout[0][rows], rows, N, True, scale,
                                             with_bound=True)
     np.testing.assert_allclose(b, eq[0][rows], rtol=1e-12, atol=0)
+
+
+# ---------------------------------------------------------------- dk / dv at selected key positions
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("H_q,H_kv", [(4, 4), (6, 2), (5, 3), (8, 1)])
+def test_kv_rows_match_full_backward(H_q, H_kv, causal):
+    # the row-selected dk/dv (score rows formed in chunks smaller than N) against the full backward
+    B, N, d, scale = 2, 29, 6, 0.45
+    q, k, v = _rand((B, N, H_q, d), 50), _rand((B, N, H_kv, d), 51), _rand((B, N, H_kv, d), 52)
+    dout = _rand((B, N, H_q, d), 53)
+    _, dk, dv = oracle.attention_backward(q, k, v, dout, causal, scale)
+    _, ek, ev = oracle.attention_backward_bound(q, k, v, dout, causal, scale)
+    rows = np.array([0, 3, 4, 17, 28, 29, 30, 44, 57])          # both batches, first and last keys
+    gk, gv, bk, bv = oracle.attention_backward_kv_rows(q, k, v, dout, rows, causal, scale, chunk=5,
+                                                       with_bound=True)
+    np.testing.assert_allclose(gk, dk.reshape(B * N, H_kv, d)[rows], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(gv, dv.reshape(B * N, H_kv, d)[rows], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(bk, ek.reshape(B * N, H_kv, d)[rows], rtol=1e-12, atol=1e-15)
+    np.testing.assert_allclose(bv, ev.reshape(B * N, H_kv, d)[rows], rtol=1e-12, atol=1e-15)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_kv_rows_match_torch_autograd(causal):
+    B, N, H_q, H_kv, d, scale = 2, 37, 6, 2, 8, 0.35
+    q, k, v = _rand((B, N, H_q, d), 54), _rand((B, N, H_kv, d), 55), _rand((B, N, H_kv, d), 56)
+    dout = _rand((B, N, H_q, d), 57)
+    R = H_q // H_kv
+    tk = torch.from_numpy(k).permute(0, 2, 1, 3).requires_grad_()
+    tv = torch.from_numpy(v).permute(0, 2, 1, 3).requires_grad_()
+    o = torch.nn.functional.scaled_dot_product_attention(
+        torch.from_numpy(q).permute(0, 2, 1, 3), tk.repeat_interleave(R, dim=1), tv.repeat_interleave(R, dim=1),
+        is_causal=causal, scale=scale)
+    o.backward(torch.from_numpy(dout).permute(0, 2, 1, 3))
+    want_k = tk.grad.permute(0, 2, 1, 3).numpy().reshape(B * N, H_kv, d)
+    want_v = tv.grad.permute(0, 2, 1, 3).numpy().reshape(B * N, H_kv, d)
+    rows = np.array([1, 2, 20, 36, 37, 50, 73])
+    gk, gv = oracle.attention_backward_kv_rows(q, k, v, dout, rows, causal, scale, chunk=8)
+    np.testing.assert_allclose(gk, want_k[rows], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(gv, want_v[rows], rtol=0, atol=1e-12)
+
+
+def test_kv_rows_planted_missing_head_is_caught(monkeypatch):
+    # a group that collects only one of its heads' shares must fail the autograd pin
+    orig = oracle.attention_backward_kv_rows
+
+    def wrong(q, k, v, dout, rows, causal, scale, chunk=128, with_bound=False):
+        R = q.shape[2] // k.shape[2]
+        keep = np.arange(q.shape[2]) % R == 0
+        return orig(q * keep[None, None, :, None], k, v, dout, rows, causal, scale, chunk, with_bound)
+    monkeypatch.setattr(oracle, "attention_backward_kv_rows", wrong)
+    with pytest.raises(AssertionError):
+        test_kv_rows_match_torch_autograd(False)

@@ -8,8 +8,10 @@ Bar: relative L2 <= 5e-3 as in the forward, and per element
 rounding-error scale of a bf16-operand backward (gradients scale with dO V^T,
 about 8 for unit-variance inputs at d = 64, so the forward's absolute 1e-2
 does not carry over). At N = 32768 dq is
-compared on >= 1024 sampled rows; dk and dv are checked through identities
-that hold at any size:
+compared on >= 1024 sampled query rows and dk, dv element by element on >= 1024
+sampled key rows (the oracle forms every score row in full for those keys'
+softmax columns); the identities below, which hold at any size, are checked
+on all of dk and dv as well:
   sum_u dV_g[u] = sum over the group's heads i of sum_t dO_i[t]   (rows of P sum to 1)
   K_g^T dK_g    = sum_i dQ_i^T Q_i                                (both are scale * Q^T dS K)
   V_g^T dV_g    = sum_i O_i^T dO_i                                (V^T P^T dO = O^T dO)
@@ -163,6 +165,15 @@ def test_backward_long_sampled(name, H_q, H_kv, d, causal):
                                                    do.reshape(B * N, H_q, d)[rows], rows, N, causal, scale,
                                                    with_bound=True)
     assert_close_bound(got, want, bound, "dq rows " + name)
+
+    kv_rows = sampled_rows(B, N, seed + 1)
+    idx_kv = torch.from_numpy(kv_rows).cuda()
+    got_k = bf16_tensor_to_f64(dk.view(B * N, H_kv, d)[idx_kv])
+    got_v = bf16_tensor_to_f64(dv.view(B * N, H_kv, d)[idx_kv])
+    want_k, want_v, bound_k, bound_v = oracle.attention_backward_kv_rows(q, k, v, do, kv_rows, causal, scale,
+                                                                         with_bound=True)
+    assert_close_bound(got_k, want_k, bound_k, "dk rows " + name)
+    assert_close_bound(got_v, want_v, bound_v, "dv rows " + name)
 
     dq64, dk64, dv64, o64 = (bf16_tensor_to_f64(x)[0] for x in (dq, dk, dv, out))
     for g in range(H_kv):

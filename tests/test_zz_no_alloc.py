@@ -75,3 +75,6 @@ def test_too_large_for_the_array_is_refused():
     assert st == sqa.SQA_ERR_WORKSPACE
     st = sqa.lib.sqa_layer_fwd_static_ws(p, p, p, p, p, p, 0, N, dm, H_q, H_kv, d, 1, ctypes.c_float(0.125), None)
     assert st == sqa.SQA_ERR_INVALID_ARG
+    # argument errors are reported as such even when the problem is also too large for the array
+    st = sqa.lib.sqa_layer_fwd_static_ws(p, p, p, p, p, p, B, N, dm, H_q, H_kv, d, 2, ctypes.c_float(0.125), None)
+    assert st == sqa.SQA_ERR_INVALID_ARG
