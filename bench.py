@@ -98,6 +98,14 @@ def load_traffic(names_hq_hkv):
     return sum(vals) / len(vals), "ncu dram__bytes_read.sum + dram__bytes_write.sum, mean per launch"
 
 
+def headline_config(world):
+    """The default workload's config object (both arms report the same one)."""
+    return {"workload": "head-config comparison, B=1 N=32768 d_head=64 non-causal "
+                        "(MHA 16/16, GQA 16/4, MQA 16/1, SQA 8/4, sSQA 8/8, xSQA 4/4, xSMQA 4/1)",
+            "global_batch": world, "seq_len": 32768, "parallelism": "dp%d" % world,
+            "l2": "flushed (256 MiB write) before every timed launch"}
+
+
 def attn_flops(B, N, H_q, d, causal):
     f = 4.0 * B * N * N * H_q * d
     return f / 2 if causal else f
@@ -327,6 +335,8 @@ def bench_sqa(args):
 
     result = None
     if rank == 0:
+        extras = headline_extras(args, sqa, torch, device, stream, peaks) if (world == 1 and not args.no_extras) \
+            else None
         cpu = cpu_baseline(seconds=args.cpu_seconds) if (world == 1 and not args.no_cpu_baseline) else None
         per = {}
         for i, c in enumerate(cfgs):
@@ -342,10 +352,7 @@ def bench_sqa(args):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(step_ms_max, 4),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded N(0,1) bf16 Q/K/V; per-rank seed)",
-            "config": {"workload": "head-config comparison, B=1 N=32768 d_head=64 non-causal "
-                                   "(MHA 16/16, GQA 16/4, MQA 16/1, SQA 8/4, sSQA 8/8, xSQA 4/4, xSMQA 4/1)",
-                       "global_batch": world, "seq_len": 32768, "parallelism": "dp%d" % world,
-                       "l2": "flushed (256 MiB write) before every timed launch"},
+            "config": headline_config(world),
             "pct_of_peak": round(100.0 * value / world / peak, 1),
             "roofline": {"bound": "tensor", "kernel": "sqa::attn_fwd_kernel<64>", "achieved": round(achieved, 1),
                          "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 3),
@@ -360,11 +367,64 @@ def bench_sqa(args):
             "speedup_vs_flop_ratio": {"t16/t8": round(t16 / t8, 3), "flop_ratio_16/8": 2.0,
                                       "t16/t4": round(t16 / t4, 3), "flop_ratio_16/4": 4.0},
             "cpu_baseline": cpu,
+            "extras": extras,
         }
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
     return result
+
+
+# ---------------------------------------------------------------------- headline extras
+SQA_CLAIM = ("up to 3x higher throughput than MHA on sequences of 32k-200k tokens, in computation-bound "
+             "scenarios (pre-training, fine-tuning, encoder tasks); hardware, model and batch not stated "
+             "(\"Sparse Query Attention (SQA)\", abstract)")
+
+
+def headline_extras(args, sqa, torch, device, stream, peaks):
+    """The rest of the metric next to the headline, each once, L2-flushed, on this GPU:
+    attention at N=200000 for MHA / SQA / xSQA (the ms-per-layer-at-200k half of the metric),
+    their speed-up over MHA beside the pages' claim, one backward, one decode step, the causal
+    layer x[4,16384,2048] and the small N=1024 case."""
+    import copy
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+    evict = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+
+    def sub(workload, steps, warmup, **kw):
+        a = copy.copy(args)
+        a.workload, a.steps, a.warmup, a.quiet = workload, steps, warmup, True
+        for key, val in kw.items():
+            setattr(a, key, val)
+        out = []
+        _bench_extra(a, sqa, torch, device, stream, flush, evict, peaks, out)
+        return out
+
+    clocks = ClockSampler(device.index or 0)
+    clocks.start()
+    try:
+        long = sub("long", 3, 1, long_N=(200000,))
+        bwd = sub("bwd", 5, 2, N=32768, hq=8, hkv=4, d=64, causal=0)
+        dec = sub("decode", 10, 3, B=8, N=32768, d=64, decode_cfgs=("MHA", "MQA"))
+        layer = sub("layer", 5, 2)
+        small = sub("small", 20, 3)
+    finally:
+        clk = clocks.stop()
+    by_hq = {(x["H_q"], x["H_kv"]): x for x in long}
+    t_mha, t_sqa, t_xsqa = (by_hq[c]["ms_median"] for c in ((16, 16), (8, 4), (4, 4)))
+    return {
+        "long_200k": {"workload": "B=1 N=200000 d_head=64 non-causal (config 3's longest length)",
+                      "per_config": {n: {k: x[k] for k in ("ms_median", "ms_min", "tflops", "pct_of_peak")}
+                                     for n, x in zip(("MHA 16/16", "SQA 8/4", "xSQA 4/4"),
+                                                     (by_hq[(16, 16)], by_hq[(8, 4)], by_hq[(4, 4)]))}},
+        "speedup_over_mha_200k": {"t_MHA/t_SQA": round(t_mha / t_sqa, 3), "flop_ratio_SQA": 2.0,
+                                  "t_MHA/t_xSQA": round(t_mha / t_xsqa, 3), "flop_ratio_xSQA": 4.0,
+                                  "pages_claim": SQA_CLAIM},
+        "backward": dict(bwd[0], note="SQA 8/4, N=32768, d=64; five N*N*d products per query head"),
+        "decode": {x["config"]: {k: x[k] for k in ("us_median", "GB_per_s", "frac_of_hbm")} for x in dec},
+        "layer": dict(layer[0], workload="causal layer x[4,16384,2048], H_q=16 H_kv=8 d=64"),
+        "small": {x["timing"]: {k: x[k] for k in ("us_median", "GB_per_s", "tflops")} for x in small},
+        "clocks": clk,
+    }
 
 
 # ---------------------------------------------------------------------- oracle timing
@@ -458,8 +518,7 @@ def bench_reference(args):
         "n_gpus": int(os.environ.get("WORLD_SIZE", "1")), "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(1e3 * s_tot / args.steps, 3), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded N(0,1) bf16 Q/K/V)",
-        "config": {"workload": "head-config comparison, B=1 N=32768 d_head=64 non-causal (sampled rows)",
-                   "global_batch": 1, "seq_len": 32768, "parallelism": "none (host cores)"},
+        "config": headline_config(int(os.environ.get("WORLD_SIZE", "1"))),
         "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -506,10 +565,15 @@ def bench_extra(args):
     return lines
 
 
+def _emit(args, line):
+    if not getattr(args, "quiet", False):
+        print(json.dumps(line), flush=True)
+
+
 def _bench_extra(args, sqa, torch, device, stream, flush, evict, peaks, lines):
     if args.workload in ("long", "sweep"):
         if args.workload == "long":
-            grid = [(N, H_q, H_kv, 64, c, 1.0, 0) for N in (65536, 131072, 200000)
+            grid = [(N, H_q, H_kv, 64, c, 1.0, 0) for N in getattr(args, "long_N", (65536, 131072, 200000))
                     for (_, H_q, H_kv) in (("MHA", 16, 16), ("SQA", 8, 4), ("xSQA", 4, 4)) for c in (0,)]
         else:
             grid = []
@@ -537,7 +601,7 @@ def _bench_extra(args, sqa, torch, device, stream, flush, evict, peaks, lines):
                           "ms_median": round(med, 3), "ms_min": round(min(ms), 3),
                           "tflops": round(fl / (med * 1e-3) / 1e12, 1),
                           "pct_of_peak": round(100 * fl / (med * 1e-3) / 1e12 / peaks["bf16_tflops"], 1)})
-            print(json.dumps(lines[-1]), flush=True)
+            _emit(args, lines[-1])
             del dev, out
     elif args.workload == "small":
         # config 1: B=1, N=1024, H_q=8, H_kv=4, d=64, non-causal, scale 1/8 -- latency-bound
@@ -567,7 +631,7 @@ def _bench_extra(args, sqa, torch, device, stream, flush, evict, peaks, lines):
             lines.append({"workload": "small", "timing": name, "us_median": round(med * 1e3, 2),
                           "us_min": round(min(ms) * 1e3, 2), "GB_per_s": round(nbytes / (med * 1e-3) / 1e9, 1),
                           "tflops": round(fl / (med * 1e-3) / 1e12, 1), "bytes": nbytes})
-            print(json.dumps(lines[-1]), flush=True)
+            _emit(args, lines[-1])
     elif args.workload == "linear":
         # one projection GEMM y[M, N_out] = x[M, K] W^T (default: the layer's QKV shape)
         import synth
@@ -591,7 +655,7 @@ def _bench_extra(args, sqa, torch, device, stream, flush, evict, peaks, lines):
         lines.append({"workload": "linear", "M": M, "K": K, "N_out": N_out, "ms_median": round(med, 4),
                       "tflops": round(fl / (med * 1e-3) / 1e12, 1),
                       "pct_of_peak": round(100 * fl / (med * 1e-3) / 1e12 / peaks["bf16_tflops"], 1)})
-        print(json.dumps(lines[-1]), flush=True)
+        _emit(args, lines[-1])
     elif args.workload == "single":
         # one attention configuration, e.g. for a profiler capture
         N, H_q, H_kv, d, causal = args.N, args.hq, args.hkv, args.d, args.causal
@@ -608,7 +672,7 @@ def _bench_extra(args, sqa, torch, device, stream, flush, evict, peaks, lines):
         med = statistics.median(ms)
         lines.append({"workload": "single", "N": N, "H_q": H_q, "H_kv": H_kv, "d": d, "causal": causal,
                       "ms_median": round(med, 3), "tflops": round(fl / (med * 1e-3) / 1e12, 1)})
-        print(json.dumps(lines[-1]), flush=True)
+        _emit(args, lines[-1])
     elif args.workload == "bwd":
         # attention backward (dq, dk, dv) at the forward's head configurations; --hq/--hkv/--d/--causal
         # given explicitly (hq != 16 or hkv != 16 or d != 64 or causal) time that one configuration instead
@@ -646,14 +710,18 @@ def _bench_extra(args, sqa, torch, device, stream, flush, evict, peaks, lines):
             lines.append({"workload": "bwd", "config": name, "N": N, "H_q": H_q, "H_kv": H_kv, "d": d,
                           "causal": causal, "ms_median": round(med, 3), "tflops": round(fl / (med * 1e-3) / 1e12, 1),
                           "pct_of_peak": round(100 * fl / (med * 1e-3) / 1e12 / peaks["bf16_tflops"], 1)})
-            print(json.dumps(lines[-1]), flush=True)
+            _emit(args, lines[-1])
             del dev, out, lse, ws, dq, dk, dv, do
     elif args.workload == "decode":
         # one new token per sequence against a 32768-token cache, the headline's head configurations;
         # memory-bound: bytes = the K/V cache (+ q and out), against the measured HBM copy bandwidth
         import synth
         B, N, d = args.B, args.N, args.d
+        wanted = getattr(args, "decode_cfgs", None)
         for name, H_q, H_kv in HEAD_CONFIGS_32K:
+            if wanted is not None and name not in wanted:
+                continue
+
             def mk(shape, tensor):
                 h = torch.empty(shape, dtype=torch.bfloat16)
                 synth.fill_bf16_into(h.data_ptr(), h.numel(), 0, tensor, 1.0)
@@ -675,7 +743,7 @@ def _bench_extra(args, sqa, torch, device, stream, flush, evict, peaks, lines):
             lines.append({"workload": "decode", "config": name, "B": B, "N": N, "H_q": H_q, "H_kv": H_kv, "d": d,
                           "us_median": round(med * 1e3, 2), "GB_per_s": round(gbs, 1),
                           "frac_of_hbm": round(gbs / peaks["hbm_gbs"], 3), "bytes": int(nbytes)})
-            print(json.dumps(lines[-1]), flush=True)
+            _emit(args, lines[-1])
             del q, k, v, out, ws
     elif args.workload == "encoder":
         # encoder-style (non-causal) layer on one long sequence, the SQA abstract's compute-bound
@@ -707,7 +775,7 @@ def _bench_extra(args, sqa, torch, device, stream, flush, evict, peaks, lines):
             lines.append({"workload": "encoder", "config": name, "N": N, "H_q": H_q, "H_kv": H_kv, "d": d,
                           "d_model": dm, "ms_per_layer": round(med, 3),
                           "tflops_total": round((fl_attn + fl_gemm) / (med * 1e-3) / 1e12, 1)})
-            print(json.dumps(lines[-1]), flush=True)
+            _emit(args, lines[-1])
             del wq, wk, wv, wo, ws
     elif args.workload == "layer":
         import synth
@@ -748,7 +816,7 @@ def _bench_extra(args, sqa, torch, device, stream, flush, evict, peaks, lines):
                       "ms_o_gemm": round(ms_o, 3),
                       "o_gemm_tflops": round(2.0 * M * (H_q * d) * dm / (ms_o * 1e-3) / 1e12, 1),
                       "ms_attention_est": round(med - ms_qkv - ms_o, 3)})
-        print(json.dumps(lines[-1]), flush=True)
+        _emit(args, lines[-1])
     return lines
 
 
@@ -772,6 +840,8 @@ def main():
     ap.add_argument("--N_out", type=int, default=2048)
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="default workload: skip the extra measurements after the headline")
     ap.add_argument("--ingest-traffic", nargs="+", default=None, metavar="CSV",
                     help="write the per-launch DRAM traffic file from ncu CSV exports, then exit")
     args = ap.parse_args()

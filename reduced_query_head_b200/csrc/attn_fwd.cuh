@@ -47,6 +47,10 @@ struct AttnParams {
   int causal;
   float scale_log2;     // scale * log2(e)
   float* lse;           // optional [B, H_q, N]: natural log of sum_u exp(scale q.k_u), or nullptr
+  // optional, layer mode: after its rows are stored, each tile adds its count of
+  // stored (token, head) rows to ready[(b * N + token) / 128] (release), for the
+  // output projection launched as this grid's programmatic dependent
+  int* ready;
   int* status;
   unsigned long long timeout_ns;
 };
@@ -93,8 +97,8 @@ struct AttnCfg {
   static_assert(!SEP_P || COL_P1 + 64 <= TMEM_COLS, "TMEM budget");
 };
 
-// EMU: of every 8 column pairs of a score row, how many take 2^x from the
-// polynomial on the FMA pipe instead of the MUFU unit (0..8).
+// EMU: bit u of this mask set = column pair u of every 8 takes 2^x from the
+// polynomial on the FMA pipe instead of the MUFU unit.
 template <int D, int EMU>
 __global__ void __launch_bounds__(384, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -112,6 +116,10 @@ __global__ void __launch_bounds__(384, 1)
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
   const int lane = tid & 31;
+  // The dependent output projection may be scheduled once every CTA of this
+  // grid has started: it then only takes SMs this grid's last wave frees, and
+  // it reads each row block only after that block's counter is complete.
+  if (p.ready != nullptr) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
   // ---- work item
   // Causal: query-tile pair outermost, longest first, so the short items fill
@@ -440,7 +448,7 @@ __global__ void __launch_bounds__(384, 1)
       for (int u = 0; u < 64; ++u) {
         const float2 x = ffma2(make_float2(s[2 * u], s[2 * u + 1]), sl2x2, nms);
         float2 e;
-        if ((u & 7) < EMU) {
+        if ((EMU >> (u & 7)) & 1) {
           e = exp2_poly2(x);
         } else {
           e.x = ex2_approx(x.x);
@@ -503,6 +511,23 @@ __global__ void __launch_bounds__(384, 1)
           uint4* d4 = reinterpret_cast<uint4*>(dst + c);
 #pragma unroll
           for (int u = 0; u < 4; ++u) d4[u] = w[u];
+        }
+      }
+      if (p.ready != nullptr) {
+        // Publish this warp's rows: each lane's stores, then one release add
+        // per 128-row block of [B * N] the warp's consecutive tokens touch
+        // (at most two).
+        __threadfence();
+        __syncwarp();
+        const long long flat = (long long)b * p.N + token;
+        const int mb = (int)(flat >> 7);
+        const int mb0 = __shfl_sync(0xffffffffu, mb, 0);
+        const unsigned in0 = __ballot_sync(0xffffffffu, store && mb == mb0);
+        const unsigned in1 = __ballot_sync(0xffffffffu, store && mb != mb0);
+        if (lane == 0) {
+          __threadfence();
+          if (in0) atomicAdd(p.ready + mb0, __popc(in0));
+          if (in1) atomicAdd(p.ready + mb0 + 1, __popc(in1));
         }
       }
     }

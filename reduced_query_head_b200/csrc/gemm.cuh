@@ -11,6 +11,14 @@
 // Persistent kernel, one CTA per SM, 128 x 256 output tiles, 64-deep K blocks
 // in a 4-stage TMA ring, two TMEM accumulators so the epilogue of one tile
 // overlaps the main loop of the next.
+//
+// Streaming X from a kernel still running (the layer's output projection):
+// with `ready` set, the kernel is launched as a programmatic dependent of the
+// attention kernel that writes X, and the producer waits, per 128-row block of
+// X, until that block's counter shows every row written (the writer adds its
+// rows with release semantics), then orders the async-proxy loads after that
+// observation. Row blocks are visited in the order the attention kernel
+// finishes them, so the projection runs on the SMs its tail frees.
 //   warp 0      TMA producer
 //   warp 1      MMA issuer + TMEM owner
 //   warps 2-5   epilogue (TMEM lane quarter = warp % 4)
@@ -29,9 +37,49 @@ struct GemmParams {
   int y_seg_start[4];
   __nv_bfloat16* y_ptr[3];
   long long y_ld[3];           // row stride (elements) of each output
+  // X written while this kernel runs: row block tm is ready once ready[tm] reaches
+  // (rows in the block) * ready_per_row; nullptr when X is complete at launch.
+  const int* ready;
+  int ready_per_row;
+  // Row-block order: 0 = natural; 1 = B batches of TB blocks each, the last
+  // block of every batch first (the order a causal longest-first attention
+  // finishes its query tiles).
+  int order, order_B, order_TB;
+  // Counters of a later kernel, zeroed by CTA 0 at start (nullptr: none).
+  int* zero_ptr;
+  int zero_count;
   int* status;
   unsigned long long timeout_ns;
 };
+
+// Row block and column block of the tile-th output tile.
+__device__ __forceinline__ void gemm_tile_coords(const GemmParams& p, int tile, int& tm, int& tn) {
+  const int mo = tile / p.tiles_n;
+  tn = tile - mo * p.tiles_n;
+  tm = p.order ? (mo % p.order_B) * p.order_TB + (p.order_TB - 1 - mo / p.order_B) : mo;
+}
+
+__device__ __forceinline__ int ld_acquire_gpu(const int* ptr) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(ptr) : "memory");
+  return v;
+}
+
+// Wait (bounded) until *ptr >= target; false on time-out or abort.
+__device__ __forceinline__ bool wait_counter(const int* ptr, int target, const WaitCtl& c) {
+  if (ld_acquire_gpu(ptr) >= target) return true;
+  const uint64_t t0 = global_timer_ns();
+  while (true) {
+    __nanosleep(128);
+    if (ld_acquire_gpu(ptr) >= target) return true;
+    if (*c.abort_flag) return false;
+    if (global_timer_ns() - t0 > c.timeout_ns) {
+      *c.abort_flag = 1;
+      atomicCAS(c.status, kStatusOk, kStatusTimeout);
+      return false;
+    }
+  }
+}
 
 struct GemmCfg {
   static constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
@@ -72,6 +120,8 @@ __global__ void __launch_bounds__(192, 1)
     *abort_flag = 0;
     fence_mbar_init();
   }
+  if (blockIdx.x == 0 && p.zero_ptr != nullptr)
+    for (int i = tid; i < p.zero_count; i += blockDim.x) p.zero_ptr[i] = 0;
   if (warp == 1) {
     tmem_alloc(smem_u32((const void*)tmem_slot), C::TMEM_COLS);
     tmem_relinquish();
@@ -90,7 +140,14 @@ __global__ void __launch_bounds__(192, 1)
       int it = 0;  // global k-block counter across tiles
       bool ok = true;
       for (int tile = blockIdx.x; ok && tile < n_tiles; tile += gridDim.x) {
-        const int tm = tile / p.tiles_n, tn = tile - tm * p.tiles_n;
+        int tm, tn;
+        gemm_tile_coords(p, tile, tm, tn);
+        if (p.ready != nullptr) {
+          // every row of this block of X written (acquire), then the async proxy may read it
+          const int rows = min(C::BM, p.M - tm * C::BM);
+          if (!wait_counter(p.ready + tm, rows * p.ready_per_row, ctl)) { ok = false; break; }
+          asm volatile("fence.proxy.async.global;" ::: "memory");
+        }
         for (int kb = 0; kb < k_blocks; ++kb, ++it) {
           const int s = it % C::STAGES;
           const int round = it / C::STAGES;
@@ -157,7 +214,8 @@ __global__ void __launch_bounds__(192, 1)
       const int use = local >> 1;
       if (!mbar_wait_warp(bar(C::BAR_ACCF + a), use & 1, ctl)) break;
       tc_fence_after();
-      const int tm = tile / p.tiles_n, tn = tile - tm * p.tiles_n;
+      int tm, tn;
+      gemm_tile_coords(p, tile, tm, tn);
       const long long row = (long long)tm * C::BM + row_in_tile;
       const bool row_ok = row < p.M;
 #pragma unroll 1

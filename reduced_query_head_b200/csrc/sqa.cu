@@ -45,12 +45,12 @@ struct DeviceState {
   int sms = 0;
 };
 
-// Attention kernels, one per head size. The template's second argument is the
-// share of exp2 evaluated by the FMA-pipe polynomial (eighths of the column
-// pairs; the rest use the MUFU unit): all-MUFU at d = 64, where the softmax
-// bounds the step, and two eighths at d = 128, where it balances the tensor work.
+// Attention kernels, one per head size. The template's second argument marks
+// the column pairs (of every 8) whose exp2 is evaluated by the FMA-pipe
+// polynomial; the rest use the MUFU unit: all-MUFU at d = 64, two eighths at
+// d = 128, where the exponentials balance the tensor work.
 using AttnKernel = void (*)(const CUtensorMap, const CUtensorMap, const CUtensorMap, const AttnParams);
-constexpr int kEmu64 = 0, kEmu128 = 2;
+constexpr int kEmu64 = 0x00, kEmu128 = 0x03;
 AttnKernel attn_kernel(int d) {
   return d == 64 ? sqa::attn_fwd_kernel<64, kEmu64> : sqa::attn_fwd_kernel<128, kEmu128>;
 }
@@ -168,7 +168,7 @@ template <int D>
 // Nk = N, the whole-sequence case).
 int launch_attn(const DeviceState* st, const void* q, const void* k, const void* v, void* out, int B, int N, int H_q,
                 int H_kv, int causal, float scale, cudaStream_t stream, float* lse = nullptr, int Nk = -1,
-                int q0 = 0) {
+                int q0 = 0, int* ready = nullptr) {
   using C = AttnCfg<D>;
   if (Nk < 0) Nk = N;
   const int P = heads_per_tile(H_q, H_kv);
@@ -222,6 +222,7 @@ int launch_attn(const DeviceState* st, const void* q, const void* k, const void*
   p.status = st->status;
   p.timeout_ns = g_wait_ns.load();
   p.lse = lse;
+  p.ready = ready;
   const AttnKernel kern = attn_kernel(D);
   kern<<<(unsigned)grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);
   return cudaGetLastError() == cudaSuccess ? SQA_OK : SQA_ERR_CUDA;
@@ -238,6 +239,13 @@ struct GemmOperands {
   int n_y;
   void* y[3];
   int y_cols[3];  // width of each output (its row stride)
+  // x written by the kernel launched just before on the same stream: this GEMM
+  // is its programmatic dependent and waits per 128-row block on `ready`
+  const int* ready = nullptr;
+  int ready_per_row = 0;
+  int order = 0, order_B = 1, order_TB = 1;   // row-block order (GemmParams)
+  int* zero_ptr = nullptr;                    // counters to zero for a later kernel
+  int zero_count = 0;
 };
 
 int launch_gemm(const DeviceState* st, const GemmOperands& g, cudaStream_t stream) {
@@ -273,16 +281,41 @@ int launch_gemm(const DeviceState* st, const GemmOperands& g, cudaStream_t strea
     p.y_ld[i] = i < g.n_y ? g.y_cols[i] : g.y_cols[0];
     if (i < g.n_y) p.y_seg_start[i + 1] = p.y_seg_start[i] + g.y_cols[i];
   }
+  p.ready = g.ready;
+  p.ready_per_row = g.ready_per_row;
+  p.order = g.order;
+  p.order_B = g.order_B;
+  p.order_TB = g.order_TB;
+  p.zero_ptr = g.zero_ptr;
+  p.zero_count = g.zero_count;
   p.status = st->status;
   p.timeout_ns = g_wait_ns.load();
   const long long tiles = (long long)p.tiles_m * p.tiles_n;
   if (tiles > INT_MAX) return SQA_ERR_INVALID_ARG;
   const int grid = (int)(tiles < st->sms ? tiles : st->sms);
-  sqa::gemm_bf16_kernel<<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tx, tw[0], tw[1], tw[2], p);
+  if (g.ready == nullptr) {
+    sqa::gemm_bf16_kernel<<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tx, tw[0], tw[1], tw[2], p);
+    return cudaGetLastError() == cudaSuccess ? SQA_OK : SQA_ERR_CUDA;
+  }
+  // programmatic dependent of the previous launch on `stream`
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3(C::THREADS);
+  cfg.dynamicSmemBytes = C::SMEM_BYTES;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, sqa::gemm_bf16_kernel, tx, tw[0], tw[1], tw[2], p) != cudaSuccess) return SQA_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? SQA_OK : SQA_ERR_CUDA;
 }
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// The layer's per-128-row-block counters of stored attention rows.
+size_t layer_ready_bytes(int B, int N) { return align256((((size_t)B * N + 127) / 128) * sizeof(int)); }
 
 // lse2 / dsum rows: a multiple of 4 floats so that every row starts 16-byte aligned.
 int bwd_row_ld(int N) { return (N + 3) & ~3; }
@@ -597,7 +630,7 @@ size_t sqa_layer_workspace_bytes(int B, int N, int d_model, int H_q, int H_kv, i
   if (B < 1 || N < 1 || d_model < 8 || H_q < 1 || H_kv < 1 || H_kv > H_q || d_head < 1) return 0;
   if (!layer_sizes_fit(B, N, d_model, H_q, H_kv, d_head)) return 0;
   const size_t M = (size_t)B * N;
-  return align256(M * H_q * d_head * 2) * 2 + align256(M * H_kv * d_head * 2) * 2;
+  return align256(M * H_q * d_head * 2) * 2 + align256(M * H_kv * d_head * 2) * 2 + layer_ready_bytes(B, N);
 }
 
 int sqa_layer_fwd(const void* x, const void* Wq, const void* Wk, const void* Wv, const void* Wo, void* out,
@@ -619,6 +652,9 @@ int sqa_layer_fwd(const void* x, const void* Wq, const void* Wk, const void* Wv,
   void* K = ws + q_bytes;
   void* V = ws + q_bytes + kv_bytes;
   void* A = ws + q_bytes + 2 * kv_bytes;
+  // one counter per 128-row block of A: rows of A the attention kernel has stored
+  int* ready = reinterpret_cast<int*>(ws + 2 * q_bytes + 2 * kv_bytes);
+  const int n_blocks = (int)((M + 127) / 128);
 
   GemmOperands g1{};
   g1.x = x;
@@ -631,10 +667,12 @@ int sqa_layer_fwd(const void* x, const void* Wq, const void* Wk, const void* Wv,
   g1.n_y = 3;
   g1.y[0] = Q; g1.y[1] = K; g1.y[2] = V;
   g1.y_cols[0] = H_q * d_head; g1.y_cols[1] = H_kv * d_head; g1.y_cols[2] = H_kv * d_head;
+  g1.zero_ptr = ready;   // zeroed before the attention kernel starts (stream order)
+  g1.zero_count = n_blocks;
   if (int e = launch_gemm(st, g1, s)) return e;
 
-  if (int e = d_head == 64 ? launch_attn<64>(st, Q, K, V, A, B, N, H_q, H_kv, causal, scale, s)
-                           : launch_attn<128>(st, Q, K, V, A, B, N, H_q, H_kv, causal, scale, s))
+  if (int e = d_head == 64 ? launch_attn<64>(st, Q, K, V, A, B, N, H_q, H_kv, causal, scale, s, nullptr, -1, 0, ready)
+                           : launch_attn<128>(st, Q, K, V, A, B, N, H_q, H_kv, causal, scale, s, nullptr, -1, 0, ready))
     return e;
 
   GemmOperands g2{};
@@ -648,6 +686,15 @@ int sqa_layer_fwd(const void* x, const void* Wq, const void* Wk, const void* Wv,
   g2.n_y = 1;
   g2.y[0] = out;
   g2.y_cols[0] = d_model;
+  // Wo consumes A's row blocks as the attention kernel completes them; causal
+  // work runs longest (latest query tiles) first, so blocks go latest first
+  g2.ready = ready;
+  g2.ready_per_row = H_q;
+  if (causal && N % 128 == 0) {
+    g2.order = 1;
+    g2.order_B = B;
+    g2.order_TB = N / 128;
+  }
   return launch_gemm(st, g2, s);
 }
 

@@ -58,6 +58,10 @@ def _run_layer(bits, B, N, dm, H_q, H_kv, d, causal, scale):
     (1, 257, 512, 8, 8, 64, False),
     (1, 200, 384, 4, 1, 128, True),
     (2, 129, 320, 6, 4, 64, True),       # uneven groups
+    (3, 512, 256, 8, 2, 64, True),       # causal, N a multiple of 128: Wo takes row blocks latest first
+    (2, 384, 256, 4, 4, 128, True),
+    (3, 200, 256, 4, 2, 64, False),      # 128-row blocks of A that straddle two sequences
+    (2, 1000, 512, 16, 2, 64, True),
 ])
 def test_layer_small_full(B, N, dm, H_q, H_kv, d, causal):
     bits = _layer_inputs(B, N, dm, H_q, H_kv, d, 13)
@@ -95,3 +99,26 @@ def test_encoder_layer_noncausal_sampled():
     f = [oracle.widen_bf16(b) for b in bits]
     want = oracle.layer_rows(f[0], f[1], f[2], f[3], f[4], rows, H_q, H_kv, d, False, 0.125, storage_rounding=True)
     assert_close(got, want, "encoder layer")
+
+
+def test_layer_repeated_calls_reuse_the_workspace():
+    """Back-to-back calls on one workspace (the row-block counters start from zero every call)
+    give the same bits; the output projection reads each block only once it is complete."""
+    import torch
+    B, N, dm, H_q, H_kv, d = 2, 640, 256, 8, 4, 64
+    bits = _layer_inputs(B, N, dm, H_q, H_kv, d, 17)
+    import reduced_query_head_b200 as sqa
+    x, wq, wk, wv, wo = (to_device_bf16(b) for b in bits)
+    ws_bytes = sqa.sqa_layer_workspace_bytes(B, N, dm, H_q, H_kv, d)
+    ws = torch.full((ws_bytes,), 0x7F, dtype=torch.uint8, device="cuda")   # garbage counters
+    outs = []
+    for _ in range(3):
+        out = torch.full((B, N, dm), float("nan"), dtype=torch.bfloat16, device="cuda")
+        sqa.sqa_layer_fwd(x, wq, wk, wv, wo, out, ws, ws_bytes, B, N, dm, H_q, H_kv, d, 1, d ** -0.5)
+        outs.append(out)
+    assert sqa.sqa_device_status() == sqa.SQA_OK
+    for o in outs[1:]:
+        assert torch.equal(o.view(torch.int16), outs[0].view(torch.int16))
+    f = [oracle.widen_bf16(b) for b in bits]
+    want = oracle.layer(f[0], f[1], f[2], f[3], f[4], H_q, H_kv, d, True, d ** -0.5, storage_rounding=True)
+    assert_close(bf16_tensor_to_f64(outs[0]), want, "layer, reused workspace", out_rounding=True)
