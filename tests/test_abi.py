@@ -75,7 +75,10 @@ def test_attn_argument_validation(sqa, args, code):
 def test_layer_workspace_size(sqa):
     B, N, dm, H_q, H_kv, d = 4, 16384, 2048, 16, 8, 64
     M = B * N
-    want = 2 * M * H_q * d * 2 + 2 * M * H_kv * d * 2
+    # Q, K, V and the attention output in bf16, then one int counter per 128-row block of the
+    # attention output (rows stored so far), rounded up to 256 bytes
+    counters = -(-(M // 128) * 4 // 256) * 256
+    want = 2 * M * H_q * d * 2 + 2 * M * H_kv * d * 2 + counters
     assert sqa.sqa_layer_workspace_bytes(B, N, dm, H_q, H_kv, d) == want
     assert sqa.sqa_layer_workspace_bytes(1, 3, 16, 2, 1, 64) % 256 == 0
     assert sqa.sqa_layer_workspace_bytes(0, 3, 16, 2, 1, 64) == 0
