@@ -42,7 +42,11 @@ struct AttnParams {
   int P, log2P;         // heads stacked per tile
   int tpt;              // tokens per 128-row tile = 128 / P
   int n_pairs;          // tile pairs per (batch, head block)
-  int n_pair_items;     // CTAs [0, n_pair_items) run two tiles; the rest run one tile each
+  // This launch runs pair items item0, item0 + 1, ...: one unit per pair, or
+  // (singles) one unit per tile of a pair. With kv_split = 2 (non-causal, a
+  // cluster of two CTAs per unit) each CTA of the cluster takes half of the
+  // key tiles and rank 1 hands its partial rows to rank 0, which merges them.
+  int item0, singles, kv_split;
   int n_hb;             // head blocks = H_q / P
   int causal;
   float scale_log2;     // scale * log2(e)
@@ -116,22 +120,27 @@ __global__ void __launch_bounds__(384, 1)
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
   const int lane = tid & 31;
-  // The dependent output projection may be scheduled once every CTA of this
-  // grid has started: it then only takes SMs this grid's last wave frees, and
-  // it reads each row block only after that block's counter is complete.
-  if (p.ready != nullptr) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  // A dependent launch (the last wave's split units, the layer's output
+  // projection) may be scheduled once every CTA of this grid has started: it
+  // then takes only SMs this grid's last wave frees. It reads nothing this grid
+  // writes, except row blocks it waits for by their counters.
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
   // ---- work item
   // Causal: query-tile pair outermost, longest first, so the short items fill
   // the tail. Non-causal: all items cost the same, so the query-tile pair is
   // innermost and CTAs running together read the same head block's K/V from L2.
-  // The last pairs of a non-causal grid may be split into one-tile CTAs so
-  // that the final wave is filled (the host decides, see n_pair_items).
-  int item = blockIdx.x, single = -1;
-  if (item >= p.n_pair_items) {
-    const int s = item - p.n_pair_items;
-    item = p.n_pair_items + (s >> 1);
-    single = s & 1;                      // which tile of the pair this CTA runs
+  // The pairs left for a last, partial wave of a non-causal grid run in a
+  // second launch whose units split the keys over two CTAs (the host decides).
+  const int split = p.kv_split;
+  const int rank = split > 1 ? (int)cluster_rank() : 0;
+  const int unit = (int)blockIdx.x / split;
+  int item, single = -1;
+  if (p.singles) {
+    item = p.item0 + (unit >> 1);
+    single = unit & 1;                   // which tile of the pair this unit runs
+  } else {
+    item = p.item0 + unit;
   }
   int qp, rest;
   if (p.causal) {
@@ -161,6 +170,16 @@ __global__ void __launch_bounds__(384, 1)
     } else {
       n_kv[k] = n_kv_all;
     }
+  }
+  // Split units (non-causal, at least two key tiles): rank 0 takes key tiles
+  // [0, half), rank 1 [half, n_kv_all).
+  int kv0 = 0;
+  if (split > 1) {
+    const int half = n_kv_all / 2;
+    kv0 = rank ? half : 0;
+#pragma unroll
+    for (int k = 0; k < 2; ++k)
+      if (n_kv[k] > 0) n_kv[k] = rank ? n_kv_all - half : half;
   }
   const int n_max = max(n_kv[0], n_kv[1]);
 
@@ -215,12 +234,12 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
         for (int c = 0; c < C::KCH; ++c)
           tma_load_4d(sbase + C::OFF_K + s * C::KV_BYTES + c * C::CHUNK_KV, &tm_k, bar(C::BAR_KF + s), c * 64, g,
-                      j * C::BN, b);
+                      (kv0 + j) * C::BN, b);
         mbar_arrive_expect_tx(bar(C::BAR_VF + s), C::KV_BYTES);
 #pragma unroll
         for (int c = 0; c < C::KCH; ++c)
           tma_load_4d(sbase + C::OFF_V + s * C::KV_BYTES + c * C::CHUNK_KV, &tm_v, bar(C::BAR_VF + s), c * 64, g,
-                      j * C::BN, b);
+                      (kv0 + j) * C::BN, b);
         filled = j + 1;
       }
       // Drain: wait (bounded) for the copies this thread issued, so none lands after exit.
@@ -415,7 +434,7 @@ __global__ void __launch_bounds__(384, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(C::BAR_SFREE + k));
 
-      const int key0 = j * C::BN;
+      const int key0 = (kv0 + j) * C::BN;
       const bool tail = key0 + C::BN > p.Nk;
       const bool diag = p.causal && (key0 + C::BN - 1 > t_first);
       if (tail || diag) {
@@ -489,24 +508,29 @@ __global__ void __launch_bounds__(384, 1)
       if (lane == 0) mbar_arrive(bar(C::BAR_P + k));
       m = m_use;
     }
-    if (ok && nk > 0 && mbar_wait_warp(bar(C::BAR_O + k), 0, ctl)) {
-      tc_fence_after();
-      const float inv_l = 1.0f / l;
-      const bool store = token < p.N;
-      // log-sum-exp of the row: l sums exp2(s*sl2 - m*sl2), so
-      // ln(sum_u exp(scale*s_u)) = (m*sl2 + log2(l)) * ln(2)
-      if (p.lse != nullptr && store)
-        p.lse[((size_t)b * p.H_q + head) * p.N + token] = (m * sl2 + __log2f(l)) * 0.69314718055994531f;
+    const bool have_o = ok && nk > 0 && mbar_wait_warp(bar(C::BAR_O + k), 0, ctl);
+    if (have_o) tc_fence_after();
+    const bool store = token < p.N;
+    // Output rows: O = (a0 * O_tmem + a1 * part) * inv_l, the row's log-sum-exp
+    // (natural log) for the backward, and the layer's row-block counters.
+    auto store_rows = [&](float a0, const float* part, float a1, float inv_l, float lse_row) {
+      if (p.lse != nullptr && store) p.lse[((size_t)b * p.H_q + head) * p.N + token] = lse_row;
       __nv_bfloat16* dst = p.out + (((size_t)b * p.N + (store ? token : 0)) * p.H_q + head) * D;
 #pragma unroll
       for (int c = 0; c < D; c += 32) {
         uint32_t r[32];
         tmem_ld32(o_addr + c, r);  // all lanes: the load is warp-collective
+        float o[32];
+#pragma unroll
+        for (int u = 0; u < 32; ++u) o[u] = __uint_as_float(r[u]) * a0;
+        if (part != nullptr) {
+#pragma unroll
+          for (int u = 0; u < 32; ++u) o[u] = fmaf(part[c + u], a1, o[u]);
+        }
         uint4 w[4];
         uint32_t* wp = reinterpret_cast<uint32_t*>(w);
 #pragma unroll
-        for (int u = 0; u < 16; ++u)
-          wp[u] = pack_bf16x2(__uint_as_float(r[2 * u]) * inv_l, __uint_as_float(r[2 * u + 1]) * inv_l);
+        for (int u = 0; u < 16; ++u) wp[u] = pack_bf16x2(o[2 * u] * inv_l, o[2 * u + 1] * inv_l);
         if (store) {
           uint4* d4 = reinterpret_cast<uint4*>(dst + c);
 #pragma unroll
@@ -530,7 +554,44 @@ __global__ void __launch_bounds__(384, 1)
           if (in1) atomicAdd(p.ready + mb0 + 1, __popc(in1));
         }
       }
+    };
+    constexpr float kLn2 = 0.69314718055994531f;
+    if (split > 1) {
+      // The two halves of the key range meet in rank 0. Partial row of tile k,
+      // row r: (D unnormalised O values, m * scale * log2(e), l) at
+      // OFF_Q + (k * 128 + r) * (D + 4) floats in rank 0's shared memory.
+      cluster_sync_all();  // both CTAs are past their main loops: rank 0's Q/K/V buffers are free
+      float* mrg = reinterpret_cast<float*>(smem + C::OFF_Q) + ((size_t)k * C::BM + row) * (D + 4);
+      if (rank == 1 && have_o) {
+        const uint32_t dst = map_shared_to_rank(smem_u32(mrg), 0);
+#pragma unroll
+        for (int c = 0; c < D; c += 32) {
+          uint32_t r[32];
+          tmem_ld32(o_addr + c, r);
+#pragma unroll
+          for (int v = 0; v < 8; ++v)
+            st_cluster_v4(dst + (c + 4 * v) * 4, __uint_as_float(r[4 * v]), __uint_as_float(r[4 * v + 1]),
+                          __uint_as_float(r[4 * v + 2]), __uint_as_float(r[4 * v + 3]));
+        }
+        st_cluster_v4(dst + D * 4, m * sl2, l, 0.f, 0.f);
+      }
+      cluster_sync_all();  // rank 1's partial rows are in rank 0's shared memory
+      if (rank == 0 && have_o) {
+        const float m0 = m * sl2, m1 = mrg[D], l1 = mrg[D + 1];
+        const float mm = fmaxf(m0, m1);
+        const float a0 = ex2_approx(m0 - mm), a1 = ex2_approx(m1 - mm);
+        const float lt = l * a0 + l1 * a1;
+        store_rows(a0, mrg, a1, 1.0f / lt, (mm + __log2f(lt)) * kLn2);
+      }
+    } else if (have_o) {
+      // l sums exp2(s*sl2 - m*sl2), so ln(sum_u exp(scale*s_u)) = (m*sl2 + log2(l)) * ln(2)
+      store_rows(1.0f, nullptr, 0.f, 1.0f / l, (m * sl2 + __log2f(l)) * kLn2);
     }
+  }
+  // Every thread of a split unit takes part in the two cluster barriers.
+  if (split > 1 && warp < 4) {
+    cluster_sync_all();
+    cluster_sync_all();
   }
 
   tc_fence_before();

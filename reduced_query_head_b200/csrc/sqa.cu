@@ -178,16 +178,27 @@ int launch_attn(const DeviceState* st, const void* q, const void* k, const void*
   const long long n_pairs = ((long long)N + 2 * tpt - 1) / (2 * tpt);
   const long long n_hb = H_q / P;
   const long long pairs = n_pairs * n_hb * B;
-  // Non-causal items all cost the same. When the pairs left over after the
-  // full waves fit in one wave as single tiles, run them that way: the last
-  // wave then finishes sooner (its softmax warps do not share MUFU units).
-  long long pair_items = pairs, grid = pairs;
+  // Non-causal items all cost the same, so the pairs left for a last, partial
+  // wave run in a second launch whose units split the keys over a cluster of
+  // two CTAs: one tile per unit when four CTAs per pair still fit in one wave
+  // (more SMs), else the whole pair per unit (two tiles per SM keep the
+  // exponential unit busier than one). Either way the last wave takes about
+  // half as long as a wave of whole pairs.
+  const long long n_kv_all = ((long long)Nk + C::BN - 1) / C::BN;
   const long long rem = pairs % st->sms;
-  if (!causal && rem > 0 && 2 * rem <= st->sms) {
-    pair_items = pairs - rem;
-    grid = pairs + rem;
+  long long main_items = pairs, tail_ctas = 0;
+  int tail_singles = 0;
+  if (!causal && rem > 0 && n_kv_all >= 2) {
+    if (4 * rem <= st->sms) {
+      main_items = pairs - rem;
+      tail_ctas = 4 * rem;
+      tail_singles = 1;
+    } else if (2 * rem <= st->sms) {
+      main_items = pairs - rem;
+      tail_ctas = 2 * rem;
+    }
   }
-  if (grid > INT_MAX) return SQA_ERR_INVALID_ARG;
+  if (pairs > INT_MAX || tail_ctas > INT_MAX) return SQA_ERR_INVALID_ARG;
 
   CUtensorMap tq, tk, tv;
   {
@@ -215,7 +226,6 @@ int launch_attn(const DeviceState* st, const void* q, const void* k, const void*
   p.log2P = log2P;
   p.tpt = tpt;
   p.n_pairs = (int)n_pairs;
-  p.n_pair_items = (int)pair_items;
   p.n_hb = (int)n_hb;
   p.causal = causal;
   p.scale_log2 = (float)((double)scale * 1.4426950408889634);  // scale * log2(e)
@@ -224,7 +234,35 @@ int launch_attn(const DeviceState* st, const void* q, const void* k, const void*
   p.lse = lse;
   p.ready = ready;
   const AttnKernel kern = attn_kernel(D);
-  kern<<<(unsigned)grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);
+  if (main_items > 0) {
+    p.item0 = 0;
+    p.singles = 0;
+    p.kv_split = 1;
+    kern<<<(unsigned)main_items, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);
+    if (cudaGetLastError() != cudaSuccess) return SQA_ERR_CUDA;
+  }
+  if (tail_ctas > 0) {
+    // clusters of two; a programmatic dependent of the main launch, so that it
+    // takes SMs as that grid's last wave frees them (it reads nothing it writes)
+    p.item0 = (int)main_items;
+    p.singles = tail_singles;
+    p.kv_split = 2;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)tail_ctas);
+    cfg.blockDim = dim3(C::THREADS);
+    cfg.dynamicSmemBytes = C::SMEM_BYTES;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = main_items > 0 ? 2 : 1;
+    if (cudaLaunchKernelEx(&cfg, kern, tq, tk, tv, p) != cudaSuccess) return SQA_ERR_CUDA;
+  }
   return cudaGetLastError() == cudaSuccess ? SQA_OK : SQA_ERR_CUDA;
 }
 

@@ -114,3 +114,24 @@ def test_config5_cost_sweep(idx, causal):
     N, H_q, H_kv = GRID[idx]
     _sampled_check(1, N, H_q, H_kv, 128, causal, seed=idx, factor=0.5,
                    what="config5 #%d N=%d Hq=%d Hkv=%d causal=%d" % (idx, N, H_q, H_kv, causal))
+
+
+# ------------------------------------------------------------ the split last wave
+# Non-causal launches whose last wave is partial run those pairs as clusters of
+# two CTAs that split the keys and merge their partial rows. Shapes that take
+# each form: one tile per unit (config 1; R = 128 with a main launch before it),
+# whole pairs per unit (H_q = 4 at N = 4096; d = 128), and none (141 pairs,
+# too many for either form in one wave).
+@pytest.mark.parametrize("shape", [(1, 1024, 8, 4, 64), (1, 640, 128, 1, 64), (1, 4096, 4, 4, 64),
+                                   (2, 1500, 4, 2, 128), (1, 9000, 4, 1, 64)],
+                         ids=lambda s: "B%dN%dHq%dHkv%dd%d" % s)
+def test_split_last_wave_full_output_and_deterministic(shape):
+    import torch
+    B, N, H_q, H_kv, d = shape
+    qb, kb, vb = attn_inputs(B, N, H_q, H_kv, d, 23)
+    a = run_attn(qb, kb, vb, False, default_scale(d))
+    b = run_attn(qb, kb, vb, False, default_scale(d))
+    assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+    want = oracle.attention(oracle.widen_bf16(qb), oracle.widen_bf16(kb), oracle.widen_bf16(vb), False,
+                            default_scale(d))
+    assert_close(bf16_tensor_to_f64(a), want, "split last wave " + str(shape), out_rounding=True)

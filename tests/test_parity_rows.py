@@ -1,9 +1,13 @@
 """GPU parity: sqa_attn_fwd_rows (a block of query rows at a global offset against all keys).
 
 Against the float64 oracle's row mode on the same seeded inputs (the forward's
-bar), and, at offsets that are multiples of the 128-row tile, bit-for-bit
-against rows of the whole-sequence sqa_attn_fwd: the shards of a sequence
-(the per-rank step of sequence sharding) reassemble the full output exactly.
+bar), and, at offsets that are multiples of the 128-row tile, against rows of
+the whole-sequence sqa_attn_fwd: the shards of a sequence (the per-rank step of
+sequence sharding) reassemble the full output within the same bar. Not bit for
+bit: a launch whose last wave is partial splits the keys of those tiles over
+two CTAs, each rounding P to bf16 against its own half's running maximum, and
+which tiles land in that wave depends on the launch's size, so a shard and the
+whole sequence can differ by P's rounding.
 """
 import numpy as np
 import pytest
@@ -52,14 +56,17 @@ def test_rows_against_oracle(case, causal):
 
 @pytest.mark.parametrize("world", [2, 4])
 @pytest.mark.parametrize("causal", [False, True])
-def test_shards_reassemble_the_whole_sequence_exactly(world, causal):
+def test_shards_reassemble_the_whole_sequence(world, causal):
     import torch
     from reduced_query_head_b200.dist import sequence_blocks
     B, N, H_q, H_kv, d = 1, 2048, 16, 4, 64
     qb, kb, vb = attn_inputs(B, N, H_q, H_kv, d, seed=71)
     full = run_attn(qb, kb, vb, causal, 0.125)
+    assembled = torch.full_like(full, float("nan"))
     for r in range(world):
         for a, b in sequence_blocks(N, r, world, causal):
             assert a % 128 == 0 and b % 128 == 0
-            part = run_rows(np.ascontiguousarray(qb[:, a:b]), kb, vb, a, causal, 0.125)
-            assert torch.equal(part.view(torch.int16), full[:, a:b].contiguous().view(torch.int16)), (r, a, b)
+            assembled[:, a:b] = run_rows(np.ascontiguousarray(qb[:, a:b]), kb, vb, a, causal, 0.125)
+    want = oracle.attention(oracle.widen_bf16(qb), oracle.widen_bf16(kb), oracle.widen_bf16(vb), causal, 0.125)
+    assert_close(bf16_tensor_to_f64(assembled), want, "sharded over %d" % world, out_rounding=True)
+    assert_close(bf16_tensor_to_f64(full), want, "whole sequence", out_rounding=True)
