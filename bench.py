@@ -64,15 +64,22 @@ def ingest_traffic(paths):
         hi = [i for i, r in enumerate(rows) if r and r[0] == "ID"][0]
         h = rows[hi]
         mi, vi, ui = h.index("Metric Name"), h.index("Metric Value"), h.index("Metric Unit")
-        unit = {"byte": 1, "Kbyte": 1e3, "Mbyte": 1e6, "Gbyte": 1e9}
-        vals = {r[mi]: float(r[vi].replace(",", "")) * unit.get(r[ui], 1) for r in rows[hi + 1:] if len(r) > vi}
+        unit = {"byte": 1, "Kbyte": 1e3, "Mbyte": 1e6, "Gbyte": 1e9, "ns": 1, "us": 1e3, "usecond": 1e3,
+                "msecond": 1e6, "nsecond": 1}
+        # one sqa_attn_fwd call may launch two grids (the split last wave): sum over the captured launches
+        vals, launches = {}, set()
+        for r in rows[hi + 1:]:
+            if len(r) > vi:
+                launches.add(r[0])
+                vals[r[mi]] = vals.get(r[mi], 0.0) + float(r[vi].replace(",", "")) * unit.get(r[ui], 1)
         per["%s/%s" % (m.group(1), m.group(2))] = {
             "dram_read_bytes": vals["dram__bytes_read.sum"], "dram_write_bytes": vals["dram__bytes_write.sum"],
-            "ncu_duration_ns": vals.get("gpu__time_duration.sum")}
+            "ncu_duration_ns": vals.get("gpu__time_duration.sum"), "launches": len(launches)}
     out = {"kernel_source_sha256": kernel_source_hash(), "per_config": per,
            "command": "ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum,gpu__time_duration.sum "
-                      "--clock-control none -k regex:attn_fwd -s 1 -c 1 --csv python bench.py --workload single "
-                      "--N 32768 --hq <H_q> --hkv <H_kv> --d 64 --steps 1 --warmup 1"}
+                      "--clock-control none -k regex:attn_fwd -s <launches per call> -c <launches per call> --csv "
+                      "python bench.py --workload single --N 32768 --hq <H_q> --hkv <H_kv> --d 64 --steps 1 "
+                      "--warmup 1 (the launches of the timed call; per-call sums)"}
     os.makedirs(os.path.dirname(TRAFFIC_FILE), exist_ok=True)
     with open(TRAFFIC_FILE, "w") as f:
         json.dump(out, f, indent=1)
@@ -361,7 +368,9 @@ def bench_sqa(args):
                          "algorithmic_bytes_per_launch": alg_bytes},
             "e2e": {"value": round(e2e_value, 2), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms_max, 4)},
-            "gpu_launches": args.steps * len(cfgs) * world,   # attention launches, all ranks
+            # attention kernel launches in the timed steps, all ranks (a call is one or two grids)
+            "gpu_launches": args.steps * world * sum(
+                sqa.sqa_attn_fwd_grids(c["B"], c["N"], c["H_q"], c["H_kv"], c["d"], 0) for c in cfgs),
             "clocks": clk,
             "per_config": per,
             "speedup_vs_flop_ratio": {"t16/t8": round(t16 / t8, 3), "flop_ratio_16/8": 2.0,

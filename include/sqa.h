@@ -96,6 +96,15 @@ int sqa_attn_fwd_rows(const void* q, const void* k, const void* v, void* out,
                       int causal, float scale, void* stream);
 
 /*
+ * Number of kernel launches sqa_attn_fwd enqueues for these sizes on the
+ * current device: 1, or 2 when the pairs of query tiles left for a partial last
+ * wave of non-causal work run in a second launch whose clusters of two CTAs
+ * split each pair's keys. 0 for invalid sizes or when the device cannot be
+ * queried. For accounting (counting launches); nothing is enqueued.
+ */
+int sqa_attn_fwd_grids(int B, int N, int H_q, int H_kv, int d_head, int causal);
+
+/*
  * Bytes of device workspace sqa_attn_bwd needs (two fp32 [B, H_q] x N row
  * arrays, rows padded to a multiple of 4 floats). Returns 0 for invalid sizes.
  */

@@ -15,7 +15,7 @@ from .build import LIB as _LIB_PATH
 __all__ = [
     "SQA_OK", "SQA_ERR_INVALID_ARG", "SQA_ERR_UNSUPPORTED", "SQA_ERR_CUDA", "SQA_ERR_TIMEOUT",
     "SQA_ERR_WORKSPACE", "SqaError", "lib", "EXPORTED_SYMBOLS", "sqa_attn_fwd", "sqa_attn_fwd_lse", "sqa_attn_fwd_rows",
-    "sqa_attn_bwd_workspace_bytes", "sqa_attn_bwd", "sqa_decode_workspace_bytes", "sqa_decode_fwd", "sqa_layer_fwd",
+    "sqa_attn_fwd_grids", "sqa_attn_bwd_workspace_bytes", "sqa_attn_bwd", "sqa_decode_workspace_bytes", "sqa_decode_fwd", "sqa_layer_fwd",
     "sqa_layer_workspace_bytes", "sqa_layer_fwd_static_ws", "SQA_STATIC_WORKSPACE_BYTES", "sqa_linear_fwd",
     "sqa_device_status", "sqa_set_wait_limit_ns",
     "sqa_check_wait_timeout", "sqa_check_exp2_poly", "sqa_status_string", "sqa_version",
@@ -25,7 +25,8 @@ SQA_OK, SQA_ERR_INVALID_ARG, SQA_ERR_UNSUPPORTED, SQA_ERR_CUDA, SQA_ERR_TIMEOUT,
 SQA_STATIC_WORKSPACE_BYTES = 64 << 20   # include/sqa.h
 
 EXPORTED_SYMBOLS = (
-    "sqa_attn_fwd", "sqa_attn_fwd_lse", "sqa_attn_fwd_rows", "sqa_attn_bwd_workspace_bytes", "sqa_attn_bwd",
+    "sqa_attn_fwd", "sqa_attn_fwd_lse", "sqa_attn_fwd_rows", "sqa_attn_fwd_grids", "sqa_attn_bwd_workspace_bytes",
+    "sqa_attn_bwd",
     "sqa_decode_workspace_bytes", "sqa_decode_fwd", "sqa_layer_workspace_bytes", "sqa_layer_fwd", "sqa_layer_fwd_static_ws", "sqa_linear_fwd",
     "sqa_device_status",
     "sqa_set_wait_limit_ns", "sqa_check_wait_timeout", "sqa_check_exp2_poly", "sqa_status_string", "sqa_version",
@@ -46,6 +47,8 @@ lib.sqa_attn_fwd_lse.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i
 lib.sqa_attn_fwd_lse.restype = _i
 lib.sqa_attn_fwd_rows.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _f, _vp]
 lib.sqa_attn_fwd_rows.restype = _i
+lib.sqa_attn_fwd_grids.argtypes = [_i, _i, _i, _i, _i, _i]
+lib.sqa_attn_fwd_grids.restype = _i
 lib.sqa_attn_bwd_workspace_bytes.argtypes = [_i, _i, _i]
 lib.sqa_attn_bwd_workspace_bytes.restype = _sz
 lib.sqa_attn_bwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _i, _i, _i, _i, _i, _i, _f, _vp]
@@ -128,6 +131,11 @@ def sqa_attn_fwd_rows(q, k, v, out, B, N_q, N_k, q_offset, H_q, H_kv, d_head, ca
     st = lib.sqa_attn_fwd_rows(_ptr(q), _ptr(k), _ptr(v), _ptr(out), B, N_q, N_k, q_offset, H_q, H_kv, d_head,
                                int(causal), float(scale), _stream(stream))
     return _check(st, "sqa_attn_fwd_rows", raise_on_error)
+
+
+def sqa_attn_fwd_grids(B, N, H_q, H_kv, d_head, causal):
+    """Kernel launches one sqa_attn_fwd call enqueues for these sizes on the current device (1 or 2; 0 if invalid)."""
+    return int(lib.sqa_attn_fwd_grids(B, N, H_q, H_kv, d_head, int(causal)))
 
 
 def sqa_attn_bwd_workspace_bytes(B, N, H_q):

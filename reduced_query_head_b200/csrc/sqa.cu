@@ -163,6 +163,42 @@ int heads_per_tile(int H_q, int H_kv) {
   return P;
 }
 
+// How one forward call covers its work: `main_items` tile pairs in one launch,
+// then (non-causal) the pairs left for a partial last wave as key-split
+// clusters of two CTAs, `tail_ctas` of them, one tile (tail_singles) or a whole
+// pair per cluster. Non-causal items all cost the same, so the pairs left for a
+// partial last wave take about half as long when their keys are split: one
+// tile per unit when four CTAs per pair still fit in one wave (more SMs), else
+// the whole pair per unit (two tiles per SM keep the exponential unit busier
+// than one).
+struct AttnPlan {
+  long long pairs, n_pairs, n_hb, main_items, tail_ctas;
+  int P, log2P, tpt, tail_singles;
+};
+AttnPlan plan_attn(int sms, int B, int N, int Nk, int H_q, int H_kv, int causal, int BM, int BN) {
+  AttnPlan a{};
+  a.P = heads_per_tile(H_q, H_kv);
+  while ((1 << a.log2P) < a.P) ++a.log2P;
+  a.tpt = BM / a.P;
+  a.n_pairs = ((long long)N + 2 * a.tpt - 1) / (2 * a.tpt);
+  a.n_hb = H_q / a.P;
+  a.pairs = a.n_pairs * a.n_hb * B;
+  const long long n_kv_all = ((long long)Nk + BN - 1) / BN;
+  const long long rem = a.pairs % sms;
+  a.main_items = a.pairs;
+  if (!causal && rem > 0 && n_kv_all >= 2) {
+    if (4 * rem <= sms) {
+      a.main_items = a.pairs - rem;
+      a.tail_ctas = 4 * rem;
+      a.tail_singles = 1;
+    } else if (2 * rem <= sms) {
+      a.main_items = a.pairs - rem;
+      a.tail_ctas = 2 * rem;
+    }
+  }
+  return a;
+}
+
 template <int D>
 // N query rows at global positions q0 .. q0 + N - 1 against Nk keys (Nk < 0:
 // Nk = N, the whole-sequence case).
@@ -171,34 +207,12 @@ int launch_attn(const DeviceState* st, const void* q, const void* k, const void*
                 int q0 = 0, int* ready = nullptr) {
   using C = AttnCfg<D>;
   if (Nk < 0) Nk = N;
-  const int P = heads_per_tile(H_q, H_kv);
-  int log2P = 0;
-  while ((1 << log2P) < P) ++log2P;
-  const int tpt = C::BM / P;
-  const long long n_pairs = ((long long)N + 2 * tpt - 1) / (2 * tpt);
-  const long long n_hb = H_q / P;
-  const long long pairs = n_pairs * n_hb * B;
-  // Non-causal items all cost the same, so the pairs left for a last, partial
-  // wave run in a second launch whose units split the keys over a cluster of
-  // two CTAs: one tile per unit when four CTAs per pair still fit in one wave
-  // (more SMs), else the whole pair per unit (two tiles per SM keep the
-  // exponential unit busier than one). Either way the last wave takes about
-  // half as long as a wave of whole pairs.
-  const long long n_kv_all = ((long long)Nk + C::BN - 1) / C::BN;
-  const long long rem = pairs % st->sms;
-  long long main_items = pairs, tail_ctas = 0;
-  int tail_singles = 0;
-  if (!causal && rem > 0 && n_kv_all >= 2) {
-    if (4 * rem <= st->sms) {
-      main_items = pairs - rem;
-      tail_ctas = 4 * rem;
-      tail_singles = 1;
-    } else if (2 * rem <= st->sms) {
-      main_items = pairs - rem;
-      tail_ctas = 2 * rem;
-    }
-  }
-  if (pairs > INT_MAX || tail_ctas > INT_MAX) return SQA_ERR_INVALID_ARG;
+  const AttnPlan plan = plan_attn(st->sms, B, N, Nk, H_q, H_kv, causal, C::BM, C::BN);
+  const int P = plan.P, log2P = plan.log2P, tpt = plan.tpt;
+  const long long n_pairs = plan.n_pairs, n_hb = plan.n_hb;
+  const long long main_items = plan.main_items, tail_ctas = plan.tail_ctas;
+  const int tail_singles = plan.tail_singles;
+  if (plan.pairs > INT_MAX || tail_ctas > INT_MAX) return SQA_ERR_INVALID_ARG;
 
   CUtensorMap tq, tk, tv;
   {
@@ -616,6 +630,16 @@ int sqa_attn_fwd_rows(const void* q, const void* k, const void* v, void* out, in
   return d_head == 64
              ? launch_attn<64>(st, q, k, v, out, B, N_q, H_q, H_kv, causal, scale, s, nullptr, N_k, q_offset)
              : launch_attn<128>(st, q, k, v, out, B, N_q, H_q, H_kv, causal, scale, s, nullptr, N_k, q_offset);
+}
+
+int sqa_attn_fwd_grids(int B, int N, int H_q, int H_kv, int d_head, int causal) {
+  if (B < 1 || N < 1 || H_q < 1 || H_kv < 1 || H_kv > H_q || (causal != 0 && causal != 1)) return 0;
+  if (d_head != 64 && d_head != 128) return 0;
+  DeviceState* st = nullptr;
+  if (device_state(&st) != SQA_OK) return 0;
+  const AttnPlan a = d_head == 64 ? plan_attn(st->sms, B, N, N, H_q, H_kv, causal, AttnCfg<64>::BM, AttnCfg<64>::BN)
+                                  : plan_attn(st->sms, B, N, N, H_q, H_kv, causal, AttnCfg<128>::BM, AttnCfg<128>::BN);
+  return (a.main_items > 0 ? 1 : 0) + (a.tail_ctas > 0 ? 1 : 0);
 }
 
 size_t sqa_attn_bwd_workspace_bytes(int B, int N, int H_q) {
