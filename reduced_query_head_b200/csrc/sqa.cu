@@ -116,15 +116,73 @@ int device_state(DeviceState** out) {
 
 bool aligned16(const void* p) { return p != nullptr && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// Tensor maps are cached per process: a map is a pure function of what it is
+// encoded from (address, data type, sizes, strides, box, swizzle, promotion),
+// so a hit returns exactly the map a fresh encode would, whatever happened to
+// the memory in between. Direct-mapped, keyed by all of those inputs; a miss
+// encodes and replaces the slot.
+struct MapKey {
+  uintptr_t base;
+  uint32_t dtype, rank, swizzle, promo;
+  cuuint64_t dims[5], strides[4];
+  cuuint32_t box[5];
+  bool operator==(const MapKey& o) const {
+    if (base != o.base || dtype != o.dtype || rank != o.rank || swizzle != o.swizzle || promo != o.promo) return false;
+    for (uint32_t i = 0; i < rank; ++i)
+      if (dims[i] != o.dims[i] || box[i] != o.box[i] || (i + 1 < rank && strides[i] != o.strides[i])) return false;
+    return true;
+  }
+};
+struct MapSlot {
+  bool used = false;
+  MapKey key;
+  CUtensorMap map;
+};
+constexpr int kMapSlots = 256;
+std::mutex g_map_mu;
+MapSlot g_maps[kMapSlots];
+
+int encode_cached(CUtensorMap* m, CUtensorMapDataType dtype, int rank, const void* base, const cuuint64_t* dims,
+                  const cuuint64_t* strides, const cuuint32_t* box, CUtensorMapSwizzle swizzle,
+                  CUtensorMapL2promotion promo) {
+  MapKey k{};
+  k.base = reinterpret_cast<uintptr_t>(base);
+  k.dtype = (uint32_t)dtype;
+  k.rank = (uint32_t)rank;
+  k.swizzle = (uint32_t)swizzle;
+  k.promo = (uint32_t)promo;
+  uint64_t h = k.base * 0x9E3779B97F4A7C15ull ^ ((uint64_t)k.dtype << 1) ^ ((uint64_t)k.swizzle << 7);
+  for (int i = 0; i < rank; ++i) {
+    k.dims[i] = dims[i];
+    k.box[i] = box[i];
+    if (i + 1 < rank) k.strides[i] = strides[i];
+    h = (h ^ (dims[i] + 0x1000193ull * box[i] + (i + 1 < rank ? strides[i] : 0))) * 0x100000001B3ull;
+  }
+  MapSlot& slot = g_maps[(h >> 32) % kMapSlots];
+  {
+    std::lock_guard<std::mutex> lk(g_map_mu);
+    if (slot.used && slot.key == k) {
+      *m = slot.map;
+      return SQA_OK;
+    }
+  }
+  const cuuint32_t es[5] = {1, 1, 1, 1, 1};
+  const CUresult r = g_encode(m, dtype, (cuuint32_t)rank, const_cast<void*>(base), dims, strides, box, es,
+                              CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, promo, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return SQA_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_map_mu);
+  slot.used = true;
+  slot.key = k;
+  slot.map = *m;
+  return SQA_OK;
+}
+
 // Tiled bf16 tensor map with 128-byte swizzle. dims/box innermost first;
 // strides in bytes for dims 1..rank-1.
 int encode_map(CUtensorMap* m, const void* base, int rank, const cuuint64_t* dims, const cuuint64_t* strides,
                const cuuint32_t* box) {
-  const cuuint32_t es[5] = {1, 1, 1, 1, 1};
-  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void*>(base), dims, strides,
-                        box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS ? SQA_OK : SQA_ERR_CUDA;
+  return encode_cached(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, base, dims, strides, box,
+                       CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B);
 }
 
 // Tiled fp32 map over `rows` rows of `cols` floats, `ld` floats apart (ld a
@@ -133,11 +191,8 @@ int encode_rows_f32(CUtensorMap* m, const float* base, long long rows, int cols,
   const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
   const cuuint64_t strides[1] = {(cuuint64_t)ld * 4};
   const cuuint32_t box[2] = {(cuuint32_t)box_cols, 1};
-  const cuuint32_t es[2] = {1, 1};
-  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(base), dims, strides, box, es,
-                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
-                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS ? SQA_OK : SQA_ERR_CUDA;
+  return encode_cached(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, base, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE,
+                       CU_TENSOR_MAP_L2_PROMOTION_L2_128B);
 }
 
 int check_attn_args(const void* q, const void* k, const void* v, const void* out, int B, int N, int H_q, int H_kv,

@@ -11,7 +11,7 @@ import pytest
 
 import oracle
 from helpers import (HEAD_CONFIGS_32K, LONG_HEAD_CONFIGS, assert_close, attn_inputs, bf16_tensor_to_f64,
-                     cost_sweep_grid, default_scale, run_attn, sampled_rows)
+                     cost_sweep_grid, default_scale, run_attn, sampled_rows, to_device_bf16)
 
 pytestmark = pytest.mark.gpu
 
@@ -135,3 +135,24 @@ def test_split_last_wave_full_output_and_deterministic(shape):
     want = oracle.attention(oracle.widen_bf16(qb), oracle.widen_bf16(kb), oracle.widen_bf16(vb), False,
                             default_scale(d))
     assert_close(bf16_tensor_to_f64(a), want, "split last wave " + str(shape), out_rounding=True)
+
+
+def test_same_buffers_different_shapes():
+    """Tensor maps are cached by address and layout: the same allocations used for another shape
+    (and then the first shape again) must give each shape's own result."""
+    import torch
+    import reduced_query_head_b200 as sqa
+    cap = 4 * 1024 * 64
+    qd = torch.empty(cap, dtype=torch.bfloat16, device="cuda")
+    kd = torch.empty(cap, dtype=torch.bfloat16, device="cuda")
+    vd = torch.empty(cap, dtype=torch.bfloat16, device="cuda")
+    od = torch.empty(cap, dtype=torch.bfloat16, device="cuda")
+    for (N, H_q, H_kv, causal) in [(1024, 4, 2, False), (512, 8, 8, True), (1024, 4, 2, False), (300, 6, 4, False)]:
+        qb, kb, vb = attn_inputs(1, N, H_q, H_kv, 64, 29)
+        for dst, src in ((qd, qb), (kd, kb), (vd, vb)):
+            dst[:src.size].copy_(to_device_bf16(src).view(-1))
+        sqa.sqa_attn_fwd(qd, kd, vd, od, 1, N, H_q, H_kv, 64, int(causal), 0.125)
+        assert sqa.sqa_device_status() == sqa.SQA_OK
+        got = bf16_tensor_to_f64(od[:N * H_q * 64].view(1, N, H_q, 64))
+        want = oracle.attention(oracle.widen_bf16(qb), oracle.widen_bf16(kb), oracle.widen_bf16(vb), causal, 0.125)
+        assert_close(got, want, "reused buffers N=%d" % N, out_rounding=True)
