@@ -72,18 +72,39 @@ def gather_sequence(local, N: int, world: int, causal: bool, group=None):
 
     `local` is [B, n_local, H, d]: this rank's rows of its sequence_blocks,
     concatenated in block order. Returns [B, N, H, d] on every rank.
+
+    One sequence (B = 1) in equal shards, the sequence-sharding case, is
+    gathered straight into the global buffer: non-causal blocks arrive in rank
+    order, which is global order; causal ranks' first chunks (0 .. world-1)
+    arrive in place, and only their second chunks (2*world-1-r, in reverse)
+    are moved once more. Other shapes go through a padded gather and a copy
+    of each block into place.
     """
     import torch
     import torch.distributed as dist
     blocks = [sequence_blocks(N, r, world, causal) for r in range(world)]
     sizes = [sum(b - a for a, b in blk) for blk in blocks]
-    top = max(sizes)
     B, n_local = local.shape[0], local.shape[1]
-    pad = torch.zeros((B, top) + tuple(local.shape[2:]), dtype=local.dtype, device=local.device)
+    rest = tuple(local.shape[2:])
+    full = torch.empty((B, N) + rest, dtype=local.dtype, device=local.device)
+    if B == 1 and len(set(sizes)) == 1 and hasattr(dist, "all_gather_into_tensor"):
+        if not causal:
+            dist.all_gather_into_tensor(full[0], local[0].contiguous(), group=group)
+            return full
+        chunk = N // (2 * world)
+        if N == 2 * world * chunk:
+            dist.all_gather_into_tensor(full[0, :world * chunk], local[0, :chunk].contiguous(), group=group)
+            late = torch.empty((world * chunk,) + rest, dtype=local.dtype, device=local.device)
+            dist.all_gather_into_tensor(late, local[0, chunk:2 * chunk].contiguous(), group=group)
+            for r in range(world):
+                c = 2 * world - 1 - r
+                full[0, c * chunk:(c + 1) * chunk] = late[r * chunk:(r + 1) * chunk]
+            return full
+    top = max(sizes)
+    pad = torch.zeros((B, top) + rest, dtype=local.dtype, device=local.device)
     pad[:, :n_local] = local
     parts = [torch.empty_like(pad) for _ in range(world)]
     dist.all_gather(parts, pad.contiguous(), group=group)
-    full = torch.empty((B, N) + tuple(local.shape[2:]), dtype=local.dtype, device=local.device)
     for r in range(world):
         off = 0
         for a, b in blocks[r]:

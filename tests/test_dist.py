@@ -105,7 +105,7 @@ def _attn_rows_cpu(q_block, k_full, v_full, q_offset, causal, scale):
     return (torch.softmax(s, dim=-1) @ v).permute(0, 2, 1, 3)
 
 
-def _seq_worker(rank, world, port, causal, q):
+def _seq_worker(rank, world, port, causal, q, B=2, N=37):
     import torch
     import torch.distributed as dist
     from reduced_query_head_b200.dist import sequence_parallel_attention
@@ -113,7 +113,7 @@ def _seq_worker(rank, world, port, causal, q):
     dist.init_process_group("gloo", rank=rank, world_size=world)
     try:
         g = torch.Generator().manual_seed(7)
-        B, N, H_q, H_kv, d, scale = 2, 37, 4, 2, 8, 0.35
+        H_q, H_kv, d, scale = 4, 2, 8, 0.35
         qf = torch.randn(B, N, H_q, d, generator=g, dtype=torch.float64)
         kf = torch.randn(B, N, H_kv, d, generator=g, dtype=torch.float64)
         vf = torch.randn(B, N, H_kv, d, generator=g, dtype=torch.float64)
@@ -127,12 +127,13 @@ def _seq_worker(rank, world, port, causal, q):
         dist.destroy_process_group()
 
 
+@pytest.mark.parametrize("B,N", [(2, 37), (1, 64)])
 @pytest.mark.parametrize("causal", [False, True])
-def test_sequence_parallel_attention_two_gloo_ranks(causal):
+def test_sequence_parallel_attention_two_gloo_ranks(causal, B, N):
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
-    procs = [ctx.Process(target=_seq_worker, args=(r, 2, port, causal, q)) for r in range(2)]
+    procs = [ctx.Process(target=_seq_worker, args=(r, 2, port, causal, q, B, N)) for r in range(2)]
     for p in procs:
         p.start()
     res = [q.get(timeout=120) for _ in procs]
@@ -141,3 +142,42 @@ def test_sequence_parallel_attention_two_gloo_ranks(causal):
         assert p.exitcode == 0
     assert sorted(r for r, _ in res) == [0, 1]
     assert max(e for _, e in res) <= 1e-12, res
+
+
+def _gather_worker(rank, world, port, cases, q):
+    import torch
+    import torch.distributed as dist
+    from reduced_query_head_b200.dist import gather_sequence
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        errs = []
+        for B, N, causal in cases:
+            full = torch.arange(B * N * 3 * 2, dtype=torch.float32).reshape(B, N, 3, 2)
+            blocks = sequence_blocks(N, rank, world, causal)
+            local = torch.cat([full[:, a:b] for a, b in blocks], dim=1)
+            got = gather_sequence(local, N, world, causal)
+            errs.append(((B, N, causal), bool(torch.equal(got, full))))
+        q.put((rank, errs))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2, 4])
+def test_gather_sequence_restores_global_order(world):
+    """The K/V exchange of sequence sharding: one sequence in equal shards (gathered straight into
+    place, causal chunks pairs included) and shapes that take the padded path (B > 1, uneven shards)."""
+    cases = [(1, 64, False), (1, 64, True), (1, 40, True), (1, 37, False), (1, 37, True), (2, 64, False),
+             (2, 37, True)]
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_gather_worker, args=(r, world, port, cases, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    res = [q.get(timeout=120) for _ in procs]
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    for _, errs in res:
+        assert all(ok for _, ok in errs), errs
