@@ -18,9 +18,10 @@
 //                         (Merging the four warps in shared memory first
 //                         measured slower: barriers and atomics per CTA.)
 //   decode_combine_kernel merges the partials of each (b, i) into out (one
-//                         CTA per head row; each thread reads a 16-column
-//                         slice of a strided set of parts). It is launched as
-//                         a programmatic dependent of the split grid, so its
+//                         CTA per head row; each thread folds a 16-column
+//                         slice of a strided set of parts into its own running
+//                         maximum, in one pass). It is launched as a
+//                         programmatic dependent of the split grid, so its
 //                         launch overlaps the split's last wave.
 #pragma once
 
@@ -282,64 +283,78 @@ __global__ void __launch_bounds__(160)
 }
 
 // One CTA of 128 threads per (b, i): merge the partials of all splits and
-// warps. Thread t owns the 16-column slice t % (D/16) of the parts
-// t / (D/16), t / (D/16) + G, ... (G part groups), so each thread keeps
-// several independent loads in flight; the groups are summed in shared memory.
+// warps in one pass. Thread t owns the 16-column slice t % (D/16) of the parts
+// t / (D/16), t / (D/16) + G, ... (G part groups) and folds them into a
+// running (max, l, o) of its own, with the loads of four parts issued before
+// any is used; the G groups' states are then merged with their own maxima.
+// Parts that saw no key hold m = -inf and weigh nothing.
 template <int D>
 __global__ void __launch_bounds__(128) decode_combine_kernel(const DecodeParams p) {
-  constexpr int CW = D / 16, G = 128 / CW;
-  __shared__ float red[128];
+  constexpr int CW = D / 16, G = 128 / CW, U = 4;
   __shared__ float gacc[G][D];
-  __shared__ float gl[G];
+  __shared__ float gm[G], gl[G];
   const int row = blockIdx.x;   // b * H_q + i
   const int t = threadIdx.x;
   // launched as a programmatic dependent of the split grid: wait until that
   // grid has completed and its partials are visible (a no-op otherwise)
   asm volatile("griddepcontrol.wait;" ::: "memory");
   const float* base = p.part + (size_t)row * p.n_parts * (D + 2);
-  // the largest partial maximum (parts that saw no key hold -inf)
-  float M = -INFINITY;
-  for (int k = t; k < p.n_parts; k += 128) M = fmaxf(M, base[(size_t)k * (D + 2)]);
-  red[t] = M;
-  __syncthreads();
-  for (int w = 64; w > 0; w >>= 1) {
-    if (t < w) red[t] = fmaxf(red[t], red[t + w]);
-    __syncthreads();
-  }
-  M = red[0];
   const int c = t % CW, pg = t / CW;
-  float acc[16];
+  float mm = -INFINITY, L = 0.f, acc[16];
 #pragma unroll
   for (int x = 0; x < 16; ++x) acc[x] = 0.f;
-  float L = 0.f;
-#pragma unroll 2
-  for (int k = pg; k < p.n_parts; k += G) {
-    const float* pk = base + (size_t)k * (D + 2);
-    const float2 ml = *reinterpret_cast<const float2*>(pk);
-    // the o slice starts 8 bytes into the 8-byte-aligned part: float2 loads
-    float v[16];
+  for (int k0 = pg; k0 < p.n_parts; k0 += U * G) {
+    float2 ml[U];
+    float v[U][16];
 #pragma unroll
-    for (int x = 0; x < 8; ++x) {
-      const float2 f2 = *reinterpret_cast<const float2*>(pk + 2 + 16 * c + 2 * x);
-      v[2 * x] = f2.x;
-      v[2 * x + 1] = f2.y;
+    for (int u = 0; u < U; ++u) {
+      const int k = k0 + u * G;
+      if (k < p.n_parts) {
+        const float* pk = base + (size_t)k * (D + 2);
+        ml[u] = *reinterpret_cast<const float2*>(pk);
+        // the o slice starts 8 bytes into the 8-byte-aligned part: float2 loads
+#pragma unroll
+        for (int x = 0; x < 8; ++x) {
+          const float2 f2 = *reinterpret_cast<const float2*>(pk + 2 + 16 * c + 2 * x);
+          v[u][2 * x] = f2.x;
+          v[u][2 * x + 1] = f2.y;
+        }
+      } else {
+        ml[u] = make_float2(-INFINITY, 0.f);
+#pragma unroll
+        for (int x = 0; x < 16; ++x) v[u][x] = 0.f;
+      }
     }
-    const float w = ex2_approx(ml.x - M);
-    L += w * ml.y;
 #pragma unroll
-    for (int x = 0; x < 16; ++x) acc[x] += w * v[x];
+    for (int u = 0; u < U; ++u) {
+      const float mn = fmaxf(mm, ml[u].x);
+      const bool any = mn != -INFINITY;
+      const float a = any ? ex2_approx(mm - mn) : 0.f;      // rescale of what is held (0 if nothing yet)
+      const float w = any ? ex2_approx(ml[u].x - mn) : 0.f;
+      L = L * a + w * ml[u].y;
+#pragma unroll
+      for (int x = 0; x < 16; ++x) acc[x] = acc[x] * a + w * v[u][x];
+      mm = mn;
+    }
   }
 #pragma unroll
   for (int x = 0; x < 16; ++x) gacc[pg][16 * c + x] = acc[x];
-  if (c == 0) gl[pg] = L;
+  if (c == 0) {
+    gm[pg] = mm;
+    gl[pg] = L;
+  }
   __syncthreads();
   if (t < D / 2) {
+    float M = -INFINITY;
+#pragma unroll 8
+    for (int g2 = 0; g2 < G; ++g2) M = fmaxf(M, gm[g2]);
     float sx = 0.f, sy = 0.f, sl = 0.f;
 #pragma unroll 4
     for (int g2 = 0; g2 < G; ++g2) {
-      sx += gacc[g2][2 * t];
-      sy += gacc[g2][2 * t + 1];
-      sl += gl[g2];
+      const float w = gm[g2] != -INFINITY ? ex2_approx(gm[g2] - M) : 0.f;
+      sx += w * gacc[g2][2 * t];
+      sy += w * gacc[g2][2 * t + 1];
+      sl += w * gl[g2];
     }
     const float inv = 1.0f / sl;
     *reinterpret_cast<uint32_t*>(p.out + (size_t)row * D + 2 * t) = pack_bf16x2(sx * inv, sy * inv);
