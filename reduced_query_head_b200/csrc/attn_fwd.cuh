@@ -600,6 +600,10 @@ __global__ void __launch_bounds__(384, 1)
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);
   }
+  // Launched as a programmatic dependent (a split last wave after its main
+  // grid), this grid must not complete before that grid: work ordered after
+  // this call on the stream relies on both. A no-op otherwise.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
 }  // namespace sqa

@@ -253,6 +253,10 @@ __global__ void __launch_bounds__(192, 1)
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);
   }
+  // Streaming mode (a programmatic dependent of the attention grid): do not
+  // complete before that grid, so work ordered after the layer on the stream
+  // finds it complete. A no-op otherwise.
+  if (p.ready != nullptr) asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
 }  // namespace sqa
