@@ -48,7 +48,8 @@ typedef enum {
   SQA_ERR_UNSUPPORTED = 2,  /* valid request this build does not implement (e.g. d_head) */
   SQA_ERR_CUDA = 3,         /* a CUDA runtime/driver call failed */
   SQA_ERR_TIMEOUT = 4,      /* a kernel wait exceeded its limit (device status) */
-  SQA_ERR_WORKSPACE = 5     /* workspace too small or misaligned */
+  SQA_ERR_WORKSPACE = 5,    /* workspace too small or misaligned */
+  SQA_ERR_BOUNDS = 6        /* debug build only: a device bounds check failed (device status) */
 } sqa_status;
 
 /*
@@ -271,6 +272,17 @@ int sqa_check_wait_timeout(unsigned long long limit_ns, void* stream);
  * SQA_ERR_INVALID_ARG otherwise. Asynchronous on `stream`.
  */
 int sqa_check_exp2_poly(const float* x, float* poly, float* ref, long long n, void* stream);
+
+/*
+ * Diagnostic of the debug build's device bounds checks (built with
+ * SQA_DEBUG_BOUNDS: every kernel checks its tile coordinates and global
+ * indices and records SQA_ERR_BOUNDS in the device status word instead of
+ * making the access). Launches one thread that evaluates a failing check with
+ * no memory access behind it, synchronises `stream`, and returns and clears
+ * the device status: SQA_ERR_BOUNDS from a debug build, SQA_OK from a release
+ * build (where the checks are compiled away).
+ */
+int sqa_check_bounds_report(void* stream);
 
 /* Human-readable name of a status code (static string). */
 const char* sqa_status_string(int status);

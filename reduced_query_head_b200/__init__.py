@@ -14,14 +14,14 @@ from .build import LIB as _LIB_PATH
 
 __all__ = [
     "SQA_OK", "SQA_ERR_INVALID_ARG", "SQA_ERR_UNSUPPORTED", "SQA_ERR_CUDA", "SQA_ERR_TIMEOUT",
-    "SQA_ERR_WORKSPACE", "SqaError", "lib", "EXPORTED_SYMBOLS", "sqa_attn_fwd", "sqa_attn_fwd_lse", "sqa_attn_fwd_rows",
+    "SQA_ERR_WORKSPACE", "SQA_ERR_BOUNDS", "SqaError", "lib", "load_debug_library", "EXPORTED_SYMBOLS", "sqa_attn_fwd", "sqa_attn_fwd_lse", "sqa_attn_fwd_rows",
     "sqa_attn_fwd_grids", "sqa_attn_bwd_workspace_bytes", "sqa_attn_bwd", "sqa_decode_workspace_bytes", "sqa_decode_fwd", "sqa_layer_fwd",
     "sqa_layer_workspace_bytes", "sqa_layer_fwd_static_ws", "SQA_STATIC_WORKSPACE_BYTES", "sqa_linear_fwd",
     "sqa_device_status", "sqa_set_wait_limit_ns",
-    "sqa_check_wait_timeout", "sqa_check_exp2_poly", "sqa_status_string", "sqa_version",
+    "sqa_check_wait_timeout", "sqa_check_exp2_poly", "sqa_check_bounds_report", "sqa_status_string", "sqa_version",
 ]
 
-SQA_OK, SQA_ERR_INVALID_ARG, SQA_ERR_UNSUPPORTED, SQA_ERR_CUDA, SQA_ERR_TIMEOUT, SQA_ERR_WORKSPACE = range(6)
+SQA_OK, SQA_ERR_INVALID_ARG, SQA_ERR_UNSUPPORTED, SQA_ERR_CUDA, SQA_ERR_TIMEOUT, SQA_ERR_WORKSPACE, SQA_ERR_BOUNDS = range(7)
 SQA_STATIC_WORKSPACE_BYTES = 64 << 20   # include/sqa.h
 
 EXPORTED_SYMBOLS = (
@@ -29,7 +29,8 @@ EXPORTED_SYMBOLS = (
     "sqa_attn_bwd",
     "sqa_decode_workspace_bytes", "sqa_decode_fwd", "sqa_layer_workspace_bytes", "sqa_layer_fwd", "sqa_layer_fwd_static_ws", "sqa_linear_fwd",
     "sqa_device_status",
-    "sqa_set_wait_limit_ns", "sqa_check_wait_timeout", "sqa_check_exp2_poly", "sqa_status_string", "sqa_version",
+    "sqa_set_wait_limit_ns", "sqa_check_wait_timeout", "sqa_check_exp2_poly", "sqa_check_bounds_report",
+    "sqa_status_string", "sqa_version",
 )
 
 if not os.path.exists(_LIB_PATH):
@@ -37,46 +38,61 @@ if not os.path.exists(_LIB_PATH):
         "libsqa.so is not built (expected at %s); run `python reduced_query_head_b200/build.py` "
         "or `python __graft_entry__.py`" % _LIB_PATH)
 
-lib = ctypes.CDLL(_LIB_PATH)
-
 _vp, _i, _f, _sz, _ll, _ull = (ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t,
                                ctypes.c_longlong, ctypes.c_ulonglong)
-lib.sqa_attn_fwd.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _vp]
-lib.sqa_attn_fwd.restype = _i
-lib.sqa_attn_fwd_lse.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _vp]
-lib.sqa_attn_fwd_lse.restype = _i
-lib.sqa_attn_fwd_rows.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _f, _vp]
-lib.sqa_attn_fwd_rows.restype = _i
-lib.sqa_attn_fwd_grids.argtypes = [_i, _i, _i, _i, _i, _i]
-lib.sqa_attn_fwd_grids.restype = _i
-lib.sqa_attn_bwd_workspace_bytes.argtypes = [_i, _i, _i]
-lib.sqa_attn_bwd_workspace_bytes.restype = _sz
-lib.sqa_attn_bwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _i, _i, _i, _i, _i, _i, _f, _vp]
-lib.sqa_attn_bwd.restype = _i
-lib.sqa_decode_workspace_bytes.argtypes = [_i, _i, _i, _i, _i]
-lib.sqa_decode_workspace_bytes.restype = _sz
-lib.sqa_decode_fwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _sz, _i, _i, _i, _i, _i, _f, _vp]
-lib.sqa_decode_fwd.restype = _i
-lib.sqa_layer_workspace_bytes.argtypes = [_i, _i, _i, _i, _i, _i]
-lib.sqa_layer_workspace_bytes.restype = _sz
-lib.sqa_layer_fwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _i, _i, _i, _i, _i, _i, _i, _f, _vp]
-lib.sqa_layer_fwd.restype = _i
-lib.sqa_layer_fwd_static_ws.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _f, _vp]
-lib.sqa_layer_fwd_static_ws.restype = _i
-lib.sqa_linear_fwd.argtypes = [_vp, _vp, _vp, _ll, _i, _i, _vp]
-lib.sqa_linear_fwd.restype = _i
-lib.sqa_device_status.argtypes = [_vp]
-lib.sqa_device_status.restype = _i
-lib.sqa_set_wait_limit_ns.argtypes = [_ull]
-lib.sqa_set_wait_limit_ns.restype = _ull
-lib.sqa_check_wait_timeout.argtypes = [_ull, _vp]
-lib.sqa_check_wait_timeout.restype = _i
-lib.sqa_check_exp2_poly.argtypes = [_vp, _vp, _vp, _ll, _vp]
-lib.sqa_check_exp2_poly.restype = _i
-lib.sqa_status_string.argtypes = [_i]
-lib.sqa_status_string.restype = ctypes.c_char_p
-lib.sqa_version.argtypes = []
-lib.sqa_version.restype = _i
+
+
+def _declare(L):
+    """Argument and result types of every entry point of a loaded libsqa."""
+    L.sqa_attn_fwd.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _vp]
+    L.sqa_attn_fwd.restype = _i
+    L.sqa_attn_fwd_lse.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _vp]
+    L.sqa_attn_fwd_lse.restype = _i
+    L.sqa_attn_fwd_rows.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _f, _vp]
+    L.sqa_attn_fwd_rows.restype = _i
+    L.sqa_attn_fwd_grids.argtypes = [_i, _i, _i, _i, _i, _i]
+    L.sqa_attn_fwd_grids.restype = _i
+    L.sqa_attn_bwd_workspace_bytes.argtypes = [_i, _i, _i]
+    L.sqa_attn_bwd_workspace_bytes.restype = _sz
+    L.sqa_attn_bwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _i, _i, _i, _i, _i, _i, _f, _vp]
+    L.sqa_attn_bwd.restype = _i
+    L.sqa_decode_workspace_bytes.argtypes = [_i, _i, _i, _i, _i]
+    L.sqa_decode_workspace_bytes.restype = _sz
+    L.sqa_decode_fwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _sz, _i, _i, _i, _i, _i, _f, _vp]
+    L.sqa_decode_fwd.restype = _i
+    L.sqa_layer_workspace_bytes.argtypes = [_i, _i, _i, _i, _i, _i]
+    L.sqa_layer_workspace_bytes.restype = _sz
+    L.sqa_layer_fwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _i, _i, _i, _i, _i, _i, _i, _f, _vp]
+    L.sqa_layer_fwd.restype = _i
+    L.sqa_layer_fwd_static_ws.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _f, _vp]
+    L.sqa_layer_fwd_static_ws.restype = _i
+    L.sqa_linear_fwd.argtypes = [_vp, _vp, _vp, _ll, _i, _i, _vp]
+    L.sqa_linear_fwd.restype = _i
+    L.sqa_device_status.argtypes = [_vp]
+    L.sqa_device_status.restype = _i
+    L.sqa_set_wait_limit_ns.argtypes = [_ull]
+    L.sqa_set_wait_limit_ns.restype = _ull
+    L.sqa_check_wait_timeout.argtypes = [_ull, _vp]
+    L.sqa_check_wait_timeout.restype = _i
+    L.sqa_check_exp2_poly.argtypes = [_vp, _vp, _vp, _ll, _vp]
+    L.sqa_check_exp2_poly.restype = _i
+    L.sqa_check_bounds_report.argtypes = [_vp]
+    L.sqa_check_bounds_report.restype = _i
+    L.sqa_status_string.argtypes = [_i]
+    L.sqa_status_string.restype = ctypes.c_char_p
+    L.sqa_version.argtypes = []
+    L.sqa_version.restype = _i
+    return L
+
+
+lib = _declare(ctypes.CDLL(_LIB_PATH))
+
+
+def load_debug_library():
+    """The debug build of the library (device bounds checks that record SQA_ERR_BOUNDS in the
+    device status word instead of faulting), built on demand, with the same entry points."""
+    from .build import build
+    return _declare(ctypes.CDLL(build(debug=True)))
 
 
 class SqaError(RuntimeError):
@@ -205,6 +221,11 @@ def sqa_check_exp2_poly(x, poly, ref, n, stream=None, raise_on_error=True):
     """poly[i] = the kernels' FMA-pipe polynomial 2^x[i], ref[i] = CUDA exp2f(x[i]) (fp32 device arrays)."""
     st = lib.sqa_check_exp2_poly(_ptr(x), _ptr(poly), _ptr(ref), int(n), _stream(stream))
     return _check(st, "sqa_check_exp2_poly", raise_on_error)
+
+
+def sqa_check_bounds_report(stream=None) -> int:
+    """SQA_ERR_BOUNDS if this library was built with device bounds checks, SQA_OK otherwise."""
+    return int(lib.sqa_check_bounds_report(_stream(stream)))
 
 
 def sqa_status_string(status: int) -> str:

@@ -225,6 +225,7 @@ __global__ void __launch_bounds__(384, 1)
         const int st = s % C::STAGES, round = s / C::STAGES;
         if (round > 0 && !mbar_wait(bar(C::BAR_EMPTY + st), (round - 1) & 1, ctl)) break;
         const int i = i0 + s / per_head, t = t_start + s % per_head;
+        if (!in_bounds(i < p.H_q && t * C::BQ < p.N && g < p.H_kv && b < p.B, p.status)) break;
         const uint32_t dst = sbase + C::OFF_STAGE + st * C::STAGE_BYTES;
         const uint32_t vec = sbase + C::OFF_VEC + st * 2 * C::VEC_BYTES;
         const uint32_t full = bar(C::BAR_FULL + st);
@@ -421,7 +422,7 @@ __global__ void __launch_bounds__(384, 1)
     // epilogue: warpgroup 0 writes dV, warpgroup 1 writes dK (x scale)
     if (ok && mbar_wait_warp(bar(C::BAR_DONE), 0, ctl) && (C::NI == 1 || mbar_wait_warp(bar(C::BAR_DONE + 1), 0, ctl))) {
       tc_fence_after();
-      const bool store = key < p.N;
+      const bool store = key < p.N && in_bounds(g < p.H_kv && b < p.B, p.status);
       const size_t base = (((size_t)b * p.N + (store ? key : 0)) * p.H_kv + g) * D;
       __nv_bfloat16* dst = (wg == 0 ? p.dv : p.dk) + base;
       const float mul = wg == 0 ? 1.0f : p.scale;
@@ -563,6 +564,7 @@ __global__ void __launch_bounds__(384, 1)
         mbar_arrive_expect_tx(bar(C::BAR_QD), 2 * C::Q_BYTES);
 #pragma unroll
         for (int c = 0; c < C::KCH; ++c) {
+          if (!in_bounds(head0 + p.P <= p.H_q && t0 < p.N && b < p.B, p.status)) break;
           tma_load_4d(sbase + C::OFF_Q + c * C::Q_CHUNK, &tm_q, bar(C::BAR_QD), c * 64, head0, t0, b);
           tma_load_4d(sbase + C::OFF_DO + c * C::Q_CHUNK, &tm_do, bar(C::BAR_QD), c * 64, head0, t0, b);
         }
@@ -571,6 +573,7 @@ __global__ void __launch_bounds__(384, 1)
       for (int j = 0; j < n_kv; ++j) {
         const int st = j % C::STAGES, round = j / C::STAGES;
         if (round > 0 && !mbar_wait(bar(C::BAR_EMPTY + st), (round - 1) & 1, ctl)) break;
+        if (!in_bounds(j * C::BK < p.N && g < p.H_kv && b < p.B, p.status)) break;
         const uint32_t dst = sbase + C::OFF_STAGE + st * C::STAGE_BYTES;
         const uint32_t full = bar(C::BAR_FULL + st);
         mbar_arrive_expect_tx(full, C::STAGE_BYTES);
@@ -771,7 +774,8 @@ __global__ void __launch_bounds__(384, 1)
                                               (!two || mbar_wait_warp(bar(C::BAR_DONE + 1), 0, ctl))));
     if (acc_ready) {
       tc_fence_after();
-      __nv_bfloat16* dst = p.dq + (((size_t)b * p.N + (row_ok ? token : 0)) * p.H_q + head) * D;
+      const bool st = row_ok && in_bounds(head < p.H_q && b < p.B, p.status);
+      __nv_bfloat16* dst = p.dq + (((size_t)b * p.N + (st ? token : 0)) * p.H_q + (st ? head : 0)) * D;
 #pragma unroll
       for (int c = wg * (D / 2); c < (wg + 1) * (D / 2); c += 32) {
         uint32_t r[32], r1[32];
@@ -787,7 +791,7 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
         for (int x = 0; x < 16; ++x)
           wp[x] = pack_bf16x2(__uint_as_float(r[2 * x]) * p.scale, __uint_as_float(r[2 * x + 1]) * p.scale);
-        if (row_ok) {
+        if (st) {
           uint4* d4 = reinterpret_cast<uint4*>(dst + c);
 #pragma unroll
           for (int x = 0; x < 4; ++x) d4[x] = w[x];

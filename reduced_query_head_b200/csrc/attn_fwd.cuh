@@ -218,18 +218,26 @@ __global__ void __launch_bounds__(384, 1)
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
-      mbar_arrive_expect_tx(bar(C::BAR_Q), 2 * C::Q_BYTES);
+      // Q of the tiles that have rows (a pair's second tile may lie past N)
+      mbar_arrive_expect_tx(bar(C::BAR_Q), ((n_kv[0] > 0) + (n_kv[1] > 0)) * C::Q_BYTES);
 #pragma unroll
-      for (int k = 0; k < 2; ++k)
+      for (int k = 0; k < 2; ++k) {
+        if (n_kv[k] == 0) continue;
 #pragma unroll
-        for (int c = 0; c < C::KCH; ++c)
+        for (int c = 0; c < C::KCH; ++c) {
+          // a failed check loads nothing: the barrier then never completes, and
+          // the waits on it end by their time limit
+          if (!in_bounds(head0 + p.P <= p.H_q && t0[k] >= 0 && t0[k] < p.N && b < p.B, p.status)) continue;
           tma_load_4d(sbase + C::OFF_Q + k * C::Q_BYTES + c * C::CHUNK_Q, &tm_q, bar(C::BAR_Q), c * 64, head0,
                       t0[k], b);
+        }
+      }
       int filled = 0;
       for (int j = 0; j < n_max; ++j) {
         const int s = j % C::STAGES;
         const int round = j / C::STAGES;
         if (round > 0 && !mbar_wait(bar(C::BAR_KVE + s), (round - 1) & 1, ctl)) break;
+        if (!in_bounds((kv0 + j) * C::BN < p.Nk && g < p.H_kv && s < C::STAGES, p.status)) break;
         mbar_arrive_expect_tx(bar(C::BAR_KF + s), C::KV_BYTES);
 #pragma unroll
         for (int c = 0; c < C::KCH; ++c)
@@ -514,8 +522,10 @@ __global__ void __launch_bounds__(384, 1)
     // Output rows: O = (a0 * O_tmem + a1 * part) * inv_l, the row's log-sum-exp
     // (natural log) for the backward, and the layer's row-block counters.
     auto store_rows = [&](float a0, const float* part, float a1, float inv_l, float lse_row) {
-      if (p.lse != nullptr && store) p.lse[((size_t)b * p.H_q + head) * p.N + token] = lse_row;
-      __nv_bfloat16* dst = p.out + (((size_t)b * p.N + (store ? token : 0)) * p.H_q + head) * D;
+      // per lane: the warp-collective TMEM loads below run on every lane either way
+      const bool st = store && in_bounds(head < p.H_q && b < p.B && token >= 0, p.status);
+      if (p.lse != nullptr && st) p.lse[((size_t)b * p.H_q + head) * p.N + token] = lse_row;
+      __nv_bfloat16* dst = p.out + (((size_t)b * p.N + (st ? token : 0)) * p.H_q + (st ? head : 0)) * D;
 #pragma unroll
       for (int c = 0; c < D; c += 32) {
         uint32_t r[32];
@@ -531,7 +541,7 @@ __global__ void __launch_bounds__(384, 1)
         uint32_t* wp = reinterpret_cast<uint32_t*>(w);
 #pragma unroll
         for (int u = 0; u < 16; ++u) wp[u] = pack_bf16x2(o[2 * u] * inv_l, o[2 * u + 1] * inv_l);
-        if (store) {
+        if (st) {
           uint4* d4 = reinterpret_cast<uint4*>(dst + c);
 #pragma unroll
           for (int u = 0; u < 4; ++u) d4[u] = w[u];
@@ -546,9 +556,10 @@ __global__ void __launch_bounds__(384, 1)
         const long long flat = (long long)b * p.N + token;
         const int mb = (int)(flat >> 7);
         const int mb0 = __shfl_sync(0xffffffffu, mb, 0);
-        const unsigned in0 = __ballot_sync(0xffffffffu, store && mb == mb0);
-        const unsigned in1 = __ballot_sync(0xffffffffu, store && mb != mb0);
-        if (lane == 0) {
+        const unsigned in0 = __ballot_sync(0xffffffffu, st && mb == mb0);
+        const unsigned in1 = __ballot_sync(0xffffffffu, st && mb != mb0);
+        const int n_blocks = (int)(((long long)p.B * p.N + 127) >> 7);
+        if (lane == 0 && (in0 | in1) != 0u && in_bounds(mb0 >= 0 && mb0 + (in1 ? 1 : 0) < n_blocks, p.status)) {
           __threadfence();
           if (in0) atomicAdd(p.ready + mb0, __popc(in0));
           if (in1) atomicAdd(p.ready + mb0 + 1, __popc(in1));
@@ -562,6 +573,7 @@ __global__ void __launch_bounds__(384, 1)
       // OFF_Q + (k * 128 + r) * (D + 4) floats in rank 0's shared memory.
       cluster_sync_all();  // both CTAs are past their main loops: rank 0's Q/K/V buffers are free
       float* mrg = reinterpret_cast<float*>(smem + C::OFF_Q) + ((size_t)k * C::BM + row) * (D + 4);
+      static_assert(C::OFF_Q + 2 * C::BM * (D + 4) * 4 <= C::OFF_BAR, "merge buffer");
       if (rank == 1 && have_o) {
         const uint32_t dst = map_shared_to_rank(smem_u32(mrg), 0);
 #pragma unroll

@@ -120,6 +120,7 @@ __global__ void __launch_bounds__(160)
       for (int j = 0; j < n_t; ++j) {
         const int st = j % C::STAGES, round = j / C::STAGES;
         if (round > 0 && !mbar_wait(bar(C::BAR_EMPTY + st), (round - 1) & 1, ctl)) break;
+        if (!in_bounds((t_begin + j) * C::BK < p.N && g < p.H_kv && b < p.B, p.status)) break;
         const uint32_t dst = sbase + st * C::STAGE_BYTES;
         const uint32_t full = bar(C::BAR_FULL + st);
         mbar_arrive_expect_tx(full, C::STAGE_BYTES);
@@ -263,7 +264,7 @@ __global__ void __launch_bounds__(160)
       lt += __shfl_xor_sync(0xffffffffu, lt, 1);
       lt += __shfl_xor_sync(0xffffffffu, lt, 2);
       const int r = h_lo + rb * 16 + g4 + 8 * half;
-      if (r < h_hi) {
+      if (r < h_hi && in_bounds(r < p.H_q && pi < p.n_parts && b < p.B, p.status)) {
         float* dst = p.part + (((size_t)b * p.H_q + r) * p.n_parts + pi) * (D + 2);
         if (t4 == 0) {
           dst[0] = m[rb][half];
@@ -357,7 +358,8 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(const DecodeParams 
       sl += w * gl[g2];
     }
     const float inv = 1.0f / sl;
-    *reinterpret_cast<uint32_t*>(p.out + (size_t)row * D + 2 * t) = pack_bf16x2(sx * inv, sy * inv);
+    if (in_bounds(row < p.B * p.H_q, p.status))
+      *reinterpret_cast<uint32_t*>(p.out + (size_t)row * D + 2 * t) = pack_bf16x2(sx * inv, sy * inv);
   }
 }
 

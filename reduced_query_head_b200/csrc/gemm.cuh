@@ -142,6 +142,7 @@ __global__ void __launch_bounds__(192, 1)
       for (int tile = blockIdx.x; ok && tile < n_tiles; tile += gridDim.x) {
         int tm, tn;
         gemm_tile_coords(p, tile, tm, tn);
+        if (!in_bounds(tm >= 0 && tm < p.tiles_m && tn >= 0 && tn < p.tiles_n, p.status)) { ok = false; break; }
         if (p.ready != nullptr) {
           // every row of this block of X written (acquire), then the async proxy may read it
           const int rows = min(C::BM, p.M - tm * C::BM);
@@ -163,6 +164,8 @@ __global__ void __launch_bounds__(192, 1)
             if (p.n_seg_w > 1 && row >= p.w_seg_start[1]) seg = 1;
             if (p.n_seg_w > 2 && row >= p.w_seg_start[2]) seg = 2;
             const void* map = seg == 0 ? (const void*)&tm_w0 : seg == 1 ? (const void*)&tm_w1 : (const void*)&tm_w2;
+            // rows past the last segment's end read as zero (a partial last N tile)
+            if (!in_bounds(row - p.w_seg_start[seg] >= 0, p.status)) continue;
             tma_load_2d(b_dst + q * 64 * 128, map, bar(C::BAR_FULL + s), kb * C::BK, row - p.w_seg_start[seg]);
           }
         }
@@ -227,6 +230,7 @@ __global__ void __launch_bounds__(192, 1)
           int seg = 0;
           if (p.n_seg_y > 1 && col >= p.y_seg_start[1]) seg = 1;
           if (p.n_seg_y > 2 && col >= p.y_seg_start[2]) seg = 2;
+          if (!in_bounds(col - p.y_seg_start[seg] + 32 <= p.y_ld[seg] || col + 32 > p.N_out, p.status)) continue;
           __nv_bfloat16* dst = p.y_ptr[seg] + row * p.y_ld[seg] + (col - p.y_seg_start[seg]);
 #pragma unroll
           for (int v = 0; v < 4; ++v) {

@@ -16,6 +16,21 @@ namespace sqa {
 
 constexpr int kStatusOk = 0;
 constexpr int kStatusTimeout = 4;
+constexpr int kStatusBounds = 6;
+
+// Debug builds (SQA_DEBUG_BOUNDS) check tile coordinates, shared-memory and
+// TMEM offsets and global indices before they are used. A failed check
+// records kStatusBounds in the device status word and the access is skipped,
+// so a bad index shows up as a status instead of a fault; other builds
+// compile the checks away.
+#ifdef SQA_DEBUG_BOUNDS
+__device__ __forceinline__ bool in_bounds(bool ok, int* status) {
+  if (!ok) atomicCAS(status, kStatusOk, kStatusBounds);
+  return ok;
+}
+#else
+__device__ __forceinline__ bool in_bounds(bool, int*) { return true; }
+#endif
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));

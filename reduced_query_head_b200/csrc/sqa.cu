@@ -650,6 +650,13 @@ int check_layer_args(const void* x, const void* Wq, const void* Wk, const void* 
   return SQA_OK;
 }
 
+// One thread evaluates a bounds check that fails, with no access behind it:
+// records SQA_ERR_BOUNDS where the checks are compiled in (debug builds).
+__global__ void bounds_probe_kernel(int* status, int n) {
+  const int idx = n;   // one past the end of an n-element range
+  sqa::in_bounds(idx < n, status);
+}
+
 }  // namespace
 
 extern "C" {
@@ -919,6 +926,15 @@ int sqa_check_exp2_poly(const float* x, float* poly, float* ref, long long n, vo
   return cudaGetLastError() == cudaSuccess ? SQA_OK : SQA_ERR_CUDA;
 }
 
+int sqa_check_bounds_report(void* stream) {
+  DeviceState* st = nullptr;
+  if (int e = device_state(&st)) return e;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  bounds_probe_kernel<<<1, 1, 0, s>>>(st->status, 16);
+  if (cudaGetLastError() != cudaSuccess) return SQA_ERR_CUDA;
+  return sqa_device_status(stream);
+}
+
 const char* sqa_status_string(int status) {
   switch (status) {
     case SQA_OK: return "SQA_OK";
@@ -927,6 +943,7 @@ const char* sqa_status_string(int status) {
     case SQA_ERR_CUDA: return "SQA_ERR_CUDA";
     case SQA_ERR_TIMEOUT: return "SQA_ERR_TIMEOUT";
     case SQA_ERR_WORKSPACE: return "SQA_ERR_WORKSPACE";
+    case SQA_ERR_BOUNDS: return "SQA_ERR_BOUNDS";
     default: return "SQA_ERR_UNKNOWN";
   }
 }

@@ -16,3 +16,4 @@ def pytest_configure(config):
     mod = importlib.util.module_from_spec(spec)
     spec.loader.exec_module(mod)
     mod.build()
+    mod.build(debug=True)

@@ -41,6 +41,14 @@ def test_library_exports_every_declared_symbol(sqa):
     assert set(_declared_functions()) == set(sqa.EXPORTED_SYMBOLS)
 
 
+def test_debug_library_exports_the_same_symbols(sqa):
+    """The bounds-checked build is the same C ABI."""
+    lib = sqa.load_debug_library()
+    for name in _declared_functions():
+        assert hasattr(lib, name), name
+    assert lib.sqa_status_string(sqa.SQA_ERR_BOUNDS) == b"SQA_ERR_BOUNDS"
+
+
 def test_status_strings_and_version(sqa):
     assert sqa.sqa_status_string(sqa.SQA_OK) == "SQA_OK"
     assert sqa.sqa_status_string(sqa.SQA_ERR_TIMEOUT) == "SQA_ERR_TIMEOUT"
