@@ -359,6 +359,7 @@ __global__ void __launch_bounds__(384, 1)
         const uint4 a = key < p.N ? s4[x] : make_uint4(0u, 0u, 0u, 0u);
         r[4 * x] = a.x; r[4 * x + 1] = a.y; r[4 * x + 2] = a.z; r[4 * x + 3] = a.w;
       }
+      __syncwarp();   // the TMEM store is warp-collective
       tmem_st32(lane_base + (wg == 0 ? C::COL_KT : C::COL_VT), r);
       tmem_st_wait();
       tc_fence_before();
@@ -430,6 +431,7 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
       for (int c = 0; c < D; c += 32) {
         uint32_t r[32];
+        __syncwarp();   // after the per-lane stores: the TMEM load is warp-collective
         tmem_ld32(col0 + c, r);
         uint4 w[4];
         uint32_t* wp = reinterpret_cast<uint32_t*>(w);
@@ -717,6 +719,7 @@ __global__ void __launch_bounds__(384, 1)
         const uint4 a = row_ok ? s4[x] : make_uint4(0u, 0u, 0u, 0u);
         r[4 * x] = a.x; r[4 * x + 1] = a.y; r[4 * x + 2] = a.z; r[4 * x + 3] = a.w;
       }
+      __syncwarp();   // the TMEM store is warp-collective
       tmem_st32(lane_base + (wg == 0 ? C::COL_QT : C::COL_DOT), r);
       tmem_st_wait();
       tc_fence_before();
@@ -779,6 +782,7 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
       for (int c = wg * (D / 2); c < (wg + 1) * (D / 2); c += 32) {
         uint32_t r[32], r1[32];
+        __syncwarp();   // after the per-lane stores: the TMEM loads are warp-collective
         if (two) {
           tmem_ld32x2(lane_base + C::COL_DQ + c, lane_base + C::COL_DQ + D + c, r, r1);
 #pragma unroll

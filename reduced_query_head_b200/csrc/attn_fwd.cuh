@@ -470,6 +470,7 @@ __global__ void __launch_bounds__(384, 1)
       const float f = (need && j > 0) ? ex2_approx((m - m_new) * sl2) : 1.0f;
       const bool rescale = (j > 0) && __any_sync(0xffffffffu, need);
       const float2 nms = make_float2(-m_use * sl2, -m_use * sl2);
+      uint32_t pk[64];
       float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
       for (int u = 0; u < 64; ++u) {
@@ -482,8 +483,12 @@ __global__ void __launch_bounds__(384, 1)
           e.y = ex2_approx(x.y);
         }
         acc[u & 3] = fadd2(acc[u & 3], e);
-        s[2 * u] = e.x;
-        s[2 * u + 1] = e.y;
+        if constexpr (C::SEP_P) {
+          pk[u] = pack_bf16x2(e.x, e.y);   // D=64: P(j) packed as it is made (+1.5%)
+        } else {
+          s[2 * u] = e.x;                  // D=128: packed at the store (packing early measured 1% slower)
+          s[2 * u + 1] = e.y;
+        }
       }
       const float2 a01 = fadd2(acc[0], acc[1]), a23 = fadd2(acc[2], acc[3]);
       const float2 a = fadd2(a01, a23);
@@ -497,7 +502,8 @@ __global__ void __launch_bounds__(384, 1)
       for (int c = 0; c < 2; ++c) {
         uint32_t r[32];
 #pragma unroll
-        for (int u = 0; u < 32; ++u) r[u] = pack_bf16x2(s[c * 64 + 2 * u], s[c * 64 + 2 * u + 1]);
+        for (int u = 0; u < 32; ++u)
+          r[u] = C::SEP_P ? pk[c * 32 + u] : pack_bf16x2(s[c * 64 + 2 * u], s[c * 64 + 2 * u + 1]);
         tmem_st32(p_addr + c * 32, r);
       }
       if (rescale) {
@@ -529,7 +535,8 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
       for (int c = 0; c < D; c += 32) {
         uint32_t r[32];
-        tmem_ld32(o_addr + c, r);  // all lanes: the load is warp-collective
+        __syncwarp();              // after the per-lane stores: the TMEM load is warp-collective
+        tmem_ld32(o_addr + c, r);
         float o[32];
 #pragma unroll
         for (int u = 0; u < 32; ++u) o[u] = __uint_as_float(r[u]) * a0;

@@ -224,6 +224,7 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll 1
       for (int c = 0; c < C::BN; c += 32) {
         uint32_t r[32];
+        __syncwarp();   // after the per-lane stores: the TMEM load is warp-collective
         tmem_ld32(lane_base + a * C::BN + c, r);
         const int col = tn * C::BN + c;
         if (row_ok && col < p.N_out) {
