@@ -431,7 +431,7 @@ def headline_extras(args, sqa, torch, device, stream, peaks):
         "backward": dict(bwd[0], note="SQA 8/4, N=32768, d=64; five N*N*d products per query head"),
         "decode": {x["config"]: {k: x[k] for k in ("us_median", "GB_per_s", "frac_of_hbm")} for x in dec},
         "layer": dict(layer[0], workload="causal layer x[4,16384,2048], H_q=16 H_kv=8 d=64"),
-        "small": {x["timing"]: {k: x[k] for k in ("us_median", "GB_per_s", "tflops")} for x in small},
+        "small": {x["timing"]: {k: x[k] for k in ("us_median", "GB_per_s", "tflops") if k in x} for x in small},
         "clocks": clk,
     }
 
@@ -640,6 +640,25 @@ def _bench_extra(args, sqa, torch, device, stream, flush, evict, peaks, lines):
             lines.append({"workload": "small", "timing": name, "us_median": round(med * 1e3, 2),
                           "us_min": round(min(ms) * 1e3, 2), "GB_per_s": round(nbytes / (med * 1e-3) / 1e9, 1),
                           "tflops": round(fl / (med * 1e-3) / 1e12, 1), "bytes": nbytes})
+            _emit(args, lines[-1])
+        # Floors of the same timing (flush, evict, events): a 4-byte torch fill (launch and
+        # event overhead alone) and this library's smallest call (one 128-row tile, one key
+        # tile: the kernel's fixed set-up, first loads and teardown).
+        tiny = torch.empty(1, dtype=torch.int32, device=device)
+        _, dev1 = make_attn_inputs(1, 128, 1, 1, d, 0, 1.0, device)
+        out1 = torch.empty((1, 128, 1, d), dtype=torch.bfloat16, device=device)
+
+        def one_tile():
+            sqa.sqa_attn_fwd(dev1["q"], dev1["k"], dev1["v"], out1, 1, 128, 1, 1, d, 0, 0.125, stream)
+        for _ in range(3):
+            tiny.fill_(0)
+            one_tile()
+        floors = (("floor_fill_4_bytes", _time_launches(lambda: tiny.fill_(0), args.steps, flush, stream, evict)),
+                  ("floor_attn_one_tile", _time_launches(one_tile, args.steps, flush, stream, evict)))
+        assert sqa.sqa_device_status(stream) == 0
+        for name, ms in floors:
+            lines.append({"workload": "small", "timing": name, "us_median": round(statistics.median(ms) * 1e3, 2),
+                          "us_min": round(min(ms) * 1e3, 2)})
             _emit(args, lines[-1])
     elif args.workload == "linear":
         # one projection GEMM y[M, N_out] = x[M, K] W^T (default: the layer's QKV shape)
