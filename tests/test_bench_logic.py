@@ -53,3 +53,44 @@ def test_order_is_near_the_best_of_all_orders():
 def test_small_counts(n):
     order = bench.pipeline_order(UP[:n], DOWN[:n], FLOPS[:n])
     assert sorted(order) == list(range(n))
+
+
+def _fake_ncu_csv(path, launches):
+    """An ncu --csv log: a preamble line, the header, then one row per (launch, metric)."""
+    import csv
+    with open(path, "w", newline="") as f:
+        f.write("==PROF== Connected to process 1\n")
+        w = csv.writer(f)
+        w.writerow(["ID", "Kernel Name", "Metric Name", "Metric Unit", "Metric Value"])
+        for i, (rd, wr, ns) in enumerate(launches):
+            w.writerow([str(i), "attn_fwd_kernel", "dram__bytes_read.sum", "Mbyte", "%.3f" % (rd / 1e6)])
+            w.writerow([str(i), "attn_fwd_kernel", "dram__bytes_write.sum", "Kbyte", "%.3f" % (wr / 1e3)])
+            w.writerow([str(i), "attn_fwd_kernel", "gpu__time_duration.sum", "usecond", "%.3f" % (ns / 1e3)])
+
+
+def test_traffic_ingest_sums_the_launches_of_a_call(tmp_path, monkeypatch):
+    """A call with a split last wave launches two grids: their counters add up per call."""
+    monkeypatch.setattr(bench, "TRAFFIC_FILE", str(tmp_path / "profiles" / "traffic.json"))
+    a = tmp_path / "traffic_16_16.csv"
+    b = tmp_path / "traffic_4_4.csv"
+    _fake_ncu_csv(str(a), [(200e6, 50e6, 5.2e6)])
+    _fake_ncu_csv(str(b), [(40e6, 1e6, 1.0e6), (20e6, 0.5e6, 0.4e6)])
+    out = bench.ingest_traffic([str(a), str(b)])
+    assert out["kernel_source_sha256"] == bench.kernel_source_hash()
+    one, two = out["per_config"]["16/16"], out["per_config"]["4/4"]
+    assert one["launches"] == 1 and two["launches"] == 2
+    assert abs(one["dram_read_bytes"] - 200e6) < 1e3 and abs(one["dram_write_bytes"] - 50e6) < 1e3
+    assert abs(two["dram_read_bytes"] - 60e6) < 1e3 and abs(two["dram_write_bytes"] - 1.5e6) < 1e3
+    assert abs(two["ncu_duration_ns"] - 1.4e6) < 1.0
+    mean, src = bench.load_traffic([(16, 16), (4, 4)])
+    assert abs(mean - (250e6 + 61.5e6) / 2) < 1e3 and "mean per launch" in src
+    assert bench.load_traffic([(8, 4)]) == (None, "config missing from capture")
+
+
+def test_traffic_from_another_kernel_build_is_not_reported(tmp_path, monkeypatch):
+    import json
+    path = tmp_path / "traffic.json"
+    monkeypatch.setattr(bench, "TRAFFIC_FILE", str(path))
+    path.write_text(json.dumps({"kernel_source_sha256": "0" * 64,
+                                "per_config": {"16/16": {"dram_read_bytes": 1.0, "dram_write_bytes": 1.0}}}))
+    assert bench.load_traffic([(16, 16)]) == (None, "capture is from an older kernel build")
