@@ -45,7 +45,7 @@ extern "C" {
 typedef enum {
   SQA_OK = 0,
   SQA_ERR_INVALID_ARG = 1,  /* null/misaligned pointer, bad size, bad scale */
-  SQA_ERR_UNSUPPORTED = 2,  /* valid request this build does not implement (e.g. d_head) */
+  SQA_ERR_UNSUPPORTED = 2,  /* valid request the library does not implement (e.g. d_head other than 64/128) */
   SQA_ERR_CUDA = 3,         /* a CUDA runtime/driver call failed */
   SQA_ERR_TIMEOUT = 4,      /* a kernel wait exceeded its limit (device status) */
   SQA_ERR_WORKSPACE = 5,    /* workspace too small or misaligned */
