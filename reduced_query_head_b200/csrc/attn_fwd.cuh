@@ -21,11 +21,15 @@
 //   warps 4-7 / 8-11  softmax for tile 0 / tile 1 (thread = row = TMEM lane):
 //            online softmax with a lazily rescaled running max, P written
 //            back to TMEM as bf16, epilogue O / l -> bf16 -> global.
-// At d=128 P is written over S, so S_k(j+1) must follow PV_k(j): one thread
-// (warp 1) issues both tiles' MMAs in the order PV_0, S_0, PV_1, S_1.
+// Each tile's S, P and O have TMEM columns of their own, so S_k(j+1) is issued
+// as soon as softmax k has read S_k(j) and overlaps softmax(j). A step takes
+// BN keys: 128 at d=64; 80 at d=128, the widest step whose S, P and O for two
+// tiles fit the 512 columns.
 //
-// TMEM columns: S0 [0,128), S1 [128,256), O0 [256,256+D), O1 [256+D,256+2D);
-// P0/P1 in [384,448)/[448,512) at d=64, over S0/S1 at d=128.
+// TMEM columns, d=64:  S0 [0,128), S1 [128,256), O0 [256,320), O1 [320,384),
+//                      P0 [384,448), P1 [448,512);
+//               d=128: S0 [0,80), P0 [80,120), S1 [128,208), P1 [208,248),
+//                      O0 [256,384), O1 [384,512).
 // Every wait is bounded; on time-out the kernel records the status, drains
 // its own copies and MMAs, frees TMEM and returns.
 #pragma once
@@ -62,16 +66,13 @@ struct AttnParams {
 template <int D>
 struct AttnCfg {
   static constexpr int BM = 128;
-  static constexpr int BN = 128;
+  static constexpr int BN = (D == 64) ? 128 : 80;      // keys per step
   static constexpr int KCH = D / 64;                    // 128-byte column chunks
-  static constexpr int STAGES = (D == 64) ? 4 : 2;
+  static constexpr int STAGES = (D == 64) ? 4 : 3;
   static constexpr int Q_BYTES = BM * D * 2;            // one Q tile
   static constexpr int KV_BYTES = BN * D * 2;           // one K (or V) tile
   static constexpr int CHUNK_Q = BM * 128;              // bytes per column chunk
   static constexpr int CHUNK_KV = BN * 128;
-  // P gets its own TMEM columns when they fit (d = 64); at d = 128 it is
-  // written over the first half of S.
-  static constexpr bool SEP_P = (D == 64);
   // shared-memory map (offsets from a 1024-aligned base)
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + 2 * Q_BYTES;
@@ -96,9 +97,12 @@ struct AttnCfg {
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr uint32_t COL_S0 = 0, COL_S1 = 128;
   static constexpr uint32_t COL_O0 = 256, COL_O1 = 256 + D;
-  static constexpr uint32_t COL_P0 = SEP_P ? 256 + 2 * D : COL_S0;
-  static constexpr uint32_t COL_P1 = SEP_P ? 256 + 2 * D + 64 : COL_S1;
-  static_assert(!SEP_P || COL_P1 + 64 <= TMEM_COLS, "TMEM budget");
+  // d=64: P0/P1 after the accumulators; d=128 (80-key steps): each P right after its S
+  static constexpr uint32_t COL_P0 = (D == 64) ? 256 + 2 * D : BN;
+  static constexpr uint32_t COL_P1 = (D == 64) ? 256 + 2 * D + 64 : 128 + BN;
+  static_assert(COL_P0 + BN / 2 <= ((D == 64) ? COL_P1 : COL_S1), "TMEM map");
+  static_assert(COL_P1 + BN / 2 <= ((D == 64) ? TMEM_COLS : COL_O0), "TMEM map");
+  static_assert(COL_O1 + D <= ((D == 64) ? COL_P0 : TMEM_COLS), "TMEM map");
 };
 
 // EMU: bit u of this mask set = column pair u of every 8 takes 2^x from the
@@ -191,7 +195,7 @@ __global__ void __launch_bounds__(384, 1)
       const bool per_warp = (i >= C::BAR_SFREE && i < C::BAR_SFREE + 2) || (i >= C::BAR_P && i < C::BAR_P + 2);
       const bool kv_empty = i >= C::BAR_KVE && i < C::BAR_KVE + C::STAGES;
       // a K/V stage is free once every MMA thread that uses it has committed it
-      mbar_init(bar(i), per_warp ? 4 : (kv_empty && C::SEP_P && active_tiles > 1) ? 2 : 1);
+      mbar_init(bar(i), per_warp ? 4 : (kv_empty && active_tiles > 1) ? 2 : 1);
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -260,80 +264,8 @@ __global__ void __launch_bounds__(384, 1)
         mbar_wait(bar(C::BAR_VF + s), (j / C::STAGES) & 1, drain);
       }
     }
-  } else if (!C::SEP_P && warp == 1) {
-    // ======================= MMA issuer (P over S): one thread, both tiles
-    // Order per step j: PV_0(j), S_0(j+1), PV_1(j), S_1(j+1). S_k(j+1) must
-    // follow PV_k(j) because P_k lives over S_k (one thread's MMAs run in
-    // issue order); the fixed order staggers the two tiles by one S + PV.
-    if (lane == 0) {
-      constexpr uint32_t IDESC_S = idesc_bf16_f32(C::BM, C::BN, 0, 0);
-      constexpr uint32_t IDESC_O = idesc_bf16_f32(C::BM, D, 0, 1);
-      // Descriptors are built once; a byte offset o inside shared memory is
-      // added as o >> 4 to the start-address field (no carry: smem < 256 KB).
-      const uint64_t dq0 = sdesc_sw128(sbase + C::OFF_Q, 16, 1024);
-      const uint64_t dk0 = sdesc_sw128(sbase + C::OFF_K, 16, 1024);
-      const uint64_t dv0 = sdesc_sw128(sbase + C::OFF_V, C::CHUNK_KV, 1024);
-      auto issue_s = [&](int k, int s) {
-        const uint64_t dq = dq0 + (uint64_t)((k * C::Q_BYTES) >> 4);
-        const uint64_t dk = dk0 + (uint64_t)((s * C::KV_BYTES) >> 4);
-        const uint32_t col_s = k ? C::COL_S1 : C::COL_S0;
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint64_t off = ((kk >> 2) * C::CHUNK_Q + (kk & 3) * 32) >> 4;
-          const uint64_t offk = ((kk >> 2) * C::CHUNK_KV + (kk & 3) * 32) >> 4;
-          umma_ss(tmem + col_s, dq + off, dk + offk, IDESC_S, kk > 0);
-        }
-      };
-      auto issue_pv = [&](int k, int s, int j) {
-        const uint64_t dv = dv0 + (uint64_t)((s * C::KV_BYTES) >> 4);
-        const uint32_t col_o = k ? C::COL_O1 : C::COL_O0;
-        const uint32_t col_p = k ? C::COL_P1 : C::COL_P0;
-#pragma unroll
-        for (int kk = 0; kk < C::BN / 16; ++kk) {
-          umma_ts(tmem + col_o, tmem + col_p + kk * 8, dv + (uint64_t)((kk * 16 * 128) >> 4), IDESC_O,
-                  (j > 0 || kk > 0) ? 1u : 0u);
-        }
-      };
-      bool ok = n_max > 0 && mbar_wait(bar(C::BAR_Q), 0, ctl) && mbar_wait(bar(C::BAR_KF + 0), 0, ctl);
-      if (ok) {
-        tc_fence_after();
-        for (int k = 0; k < 2; ++k)
-          if (n_kv[k] > 0) {
-            issue_s(k, 0);
-            umma_commit(bar(C::BAR_S + k));
-          }
-      }
-      for (int j = 0; ok && j < n_max; ++j) {
-        const int s = j % C::STAGES;
-        const uint32_t ph = (j / C::STAGES) & 1;
-        const int s1 = (j + 1) % C::STAGES;
-        const uint32_t ph1 = ((j + 1) / C::STAGES) & 1;
-        if (!mbar_wait(bar(C::BAR_VF + s), ph, ctl)) { ok = false; break; }
-        for (int k = 0; k < 2 && ok; ++k) {
-          if (j >= n_kv[k]) continue;
-          if (!mbar_wait(bar(C::BAR_P + k), j & 1, ctl)) { ok = false; break; }
-          tc_fence_after();
-          issue_pv(k, s, j);
-          umma_commit(bar(C::BAR_PV + k));
-          if (j == n_kv[k] - 1) {
-            umma_commit(bar(C::BAR_O + k));
-          } else {
-            if (!mbar_wait(bar(C::BAR_KF + s1), ph1, ctl)) { ok = false; break; }
-            tc_fence_after();
-            issue_s(k, s1);
-            umma_commit(bar(C::BAR_S + k));
-          }
-        }
-        umma_commit(bar(C::BAR_KVE + s));
-      }
-      // Drain: every MMA issued above has finished before TMEM is released.
-      umma_commit(bar(C::BAR_DRAIN));
-      volatile int zero = 0;
-      WaitCtl drain{&zero, p.status, drain_limit_ns(p.timeout_ns)};
-      mbar_wait(bar(C::BAR_DRAIN), 0, drain);
-    }
-  } else if (C::SEP_P && (warp == 1 || warp == 3)) {
-    // ======================= MMA issuers (P in its own columns): one thread per tile
+  } else if (warp == 1 || warp == 3) {
+    // ======================= MMA issuers: one thread per tile
     // Each tile's S/PV chain runs on its own thread, so a slow step of one
     // tile never holds up the other (issue blocks until the tensor core
     // accepts the MMA). Both threads feed the same tensor core; they touch
@@ -346,7 +278,8 @@ __global__ void __launch_bounds__(384, 1)
       const uint32_t col_o = k ? C::COL_O1 : C::COL_O0;
       const uint32_t col_p = k ? C::COL_P1 : C::COL_P0;
       const int nk = n_kv[k];
-      // descriptors built once; offsets added as o >> 4 (see the D = 128 path)
+      // Descriptors are built once; a byte offset o inside shared memory is
+      // added as o >> 4 to the start-address field (no carry: smem < 256 KB).
       const uint64_t dq = sdesc_sw128(sbase + C::OFF_Q + k * C::Q_BYTES, 16, 1024);
       const uint64_t dk0 = sdesc_sw128(sbase + C::OFF_K, 16, 1024);
       const uint64_t dv0 = sdesc_sw128(sbase + C::OFF_V, C::CHUNK_KV, 1024);
@@ -430,12 +363,22 @@ __global__ void __launch_bounds__(384, 1)
     for (int j = 0; j < nk; ++j) {
       if (!mbar_wait_warp(bar(C::BAR_S + k), j & 1, ctl)) { ok = false; break; }
       tc_fence_after();
-      float s[128];
-      {
+      constexpr int NC = C::BN;
+      float s[NC];
+      if constexpr (NC == 128) {
         uint32_t r[128];
         tmem_ld128(s_addr, r);
 #pragma unroll
         for (int u = 0; u < 128; ++u) s[u] = __uint_as_float(r[u]);
+      } else {
+        static_assert(NC == 80, "score columns");
+        uint32_t r[64], r2[16];
+        tmem_ld64(s_addr, r);
+        tmem_ld16(s_addr + 64, r2);
+#pragma unroll
+        for (int u = 0; u < 64; ++u) s[u] = __uint_as_float(r[u]);
+#pragma unroll
+        for (int u = 0; u < 16; ++u) s[64 + u] = __uint_as_float(r2[u]);
       }
       // S_k is in registers: the next S_k may be written.
       tc_fence_before();
@@ -448,7 +391,7 @@ __global__ void __launch_bounds__(384, 1)
       if (tail || diag) {
         const int lim = p.causal ? min(p.q0 + token, p.Nk - 1) : p.Nk - 1;  // last visible key
 #pragma unroll
-        for (int u = 0; u < 128; ++u)
+        for (int u = 0; u < NC; ++u)
           if (key0 + u > lim) s[u] = -INFINITY;
       }
       // row maximum: eight independent 3-input chains, then a short tree
@@ -456,11 +399,11 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
       for (int i = 0; i < 8; ++i) m8[i] = fmax3(s[i], s[8 + i], s[16 + i]);
 #pragma unroll
-      for (int u = 24; u < 120; u += 16)
+      for (int u = 24; u < NC - 8; u += 16)
 #pragma unroll
         for (int i = 0; i < 8; ++i) m8[i] = fmax3(m8[i], s[u + i], s[u + 8 + i]);
 #pragma unroll
-      for (int i = 0; i < 8; ++i) m8[i] = fmaxf(m8[i], s[120 + i]);
+      for (int i = 0; i < 8; ++i) m8[i] = fmaxf(m8[i], s[NC - 8 + i]);
       const float mx = fmax3(fmax3(m8[0], m8[1], m8[2]), fmax3(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7]));
       const float m_new = fmaxf(m, mx);
       // Keep the stale maximum unless it grew by more than 2^8 in the exp2
@@ -470,10 +413,10 @@ __global__ void __launch_bounds__(384, 1)
       const float f = (need && j > 0) ? ex2_approx((m - m_new) * sl2) : 1.0f;
       const bool rescale = (j > 0) && __any_sync(0xffffffffu, need);
       const float2 nms = make_float2(-m_use * sl2, -m_use * sl2);
-      uint32_t pk[64];
+      uint32_t pk[NC / 2];
       float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
-      for (int u = 0; u < 64; ++u) {
+      for (int u = 0; u < NC / 2; ++u) {
         const float2 x = ffma2(make_float2(s[2 * u], s[2 * u + 1]), sl2x2, nms);
         float2 e;
         if ((EMU >> (u & 7)) & 1) {
@@ -483,12 +426,7 @@ __global__ void __launch_bounds__(384, 1)
           e.y = ex2_approx(x.y);
         }
         acc[u & 3] = fadd2(acc[u & 3], e);
-        if constexpr (C::SEP_P) {
-          pk[u] = pack_bf16x2(e.x, e.y);   // D=64: P(j) packed as it is made (+1.5%)
-        } else {
-          s[2 * u] = e.x;                  // D=128: packed at the store (packing early measured 1% slower)
-          s[2 * u + 1] = e.y;
-        }
+        pk[u] = pack_bf16x2(e.x, e.y);   // P(j) packed as it is made
       }
       const float2 a01 = fadd2(acc[0], acc[1]), a23 = fadd2(acc[2], acc[3]);
       const float2 a = fadd2(a01, a23);
@@ -498,13 +436,22 @@ __global__ void __launch_bounds__(384, 1)
         if (!mbar_wait_warp(bar(C::BAR_PV + k), (j - 1) & 1, ctl)) { ok = false; break; }
         tc_fence_after();
       }
+      if constexpr (NC == 128) {
 #pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        uint32_t r[32];
+        for (int c = 0; c < 2; ++c) {
+          uint32_t r[32];
 #pragma unroll
-        for (int u = 0; u < 32; ++u)
-          r[u] = C::SEP_P ? pk[c * 32 + u] : pack_bf16x2(s[c * 64 + 2 * u], s[c * 64 + 2 * u + 1]);
-        tmem_st32(p_addr + c * 32, r);
+          for (int u = 0; u < 32; ++u) r[u] = pk[c * 32 + u];
+          tmem_st32(p_addr + c * 32, r);
+        }
+      } else {
+        uint32_t r[32], r8[8];
+#pragma unroll
+        for (int u = 0; u < 32; ++u) r[u] = pk[u];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) r8[u] = pk[32 + u];
+        tmem_st32(p_addr, r);
+        tmem_st8(p_addr + 32, r8);
       }
       if (rescale) {
 #pragma unroll 1
