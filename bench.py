@@ -393,8 +393,8 @@ SQA_CLAIM = ("up to 3x higher throughput than MHA on sequences of 32k-200k token
 def headline_extras(args, sqa, torch, device, stream, peaks):
     """The rest of the metric next to the headline, each once, L2-flushed, on this GPU:
     attention at N=200000 for MHA / SQA / xSQA (the ms-per-layer-at-200k half of the metric),
-    their speed-up over MHA beside the pages' claim, one backward, one decode step, the causal
-    layer x[4,16384,2048] and the small N=1024 case."""
+    their speed-up over MHA beside the pages' claim, four d=128 points of the cost sweep, one
+    backward, one decode step, the causal layer x[4,16384,2048] and the small N=1024 case."""
     import copy
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
     evict = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
@@ -412,6 +412,8 @@ def headline_extras(args, sqa, torch, device, stream, peaks):
     clocks.start()
     try:
         long = sub("long", 3, 1, long_N=(200000,))
+        d128 = sub("sweep", 3, 1, sweep_points={(32768, 32, 8, 0), (32768, 32, 8, 1), (65536, 16, 4, 0),
+                                                (65536, 16, 4, 1)})
         bwd = sub("bwd", 5, 2, N=32768, hq=8, hkv=4, d=64, causal=0)
         dec = sub("decode", 10, 3, B=8, N=32768, d=64, decode_cfgs=("MHA", "MQA"))
         layer = sub("layer", 5, 2)
@@ -428,6 +430,12 @@ def headline_extras(args, sqa, torch, device, stream, peaks):
         "speedup_over_mha_200k": {"t_MHA/t_SQA": round(t_mha / t_sqa, 3), "flop_ratio_SQA": 2.0,
                                   "t_MHA/t_xSQA": round(t_mha / t_xsqa, 3), "flop_ratio_xSQA": 4.0,
                                   "pages_claim": SQA_CLAIM},
+        "d128_sweep_points": {
+            "workload": "config 5 points (cost sweep, d_head=128, inputs x0.5, seed = grid index); the full "
+                        "88-point sweep is --workload sweep",
+            "per_point": {"N=%d H_q=%d H_kv=%d %s" % (x["N"], x["H_q"], x["H_kv"], "causal" if x["causal"] else
+                                                      "non-causal"):
+                          {k: x[k] for k in ("ms_median", "tflops", "pct_of_peak")} for x in d128}},
         "backward": dict(bwd[0], note="SQA 8/4, N=32768, d=64; five N*N*d products per query head"),
         "decode": {x["config"]: {k: x[k] for k in ("us_median", "GB_per_s", "frac_of_hbm")} for x in dec},
         "layer": dict(layer[0], workload="causal layer x[4,16384,2048], H_q=16 H_kv=8 d=64"),
@@ -594,6 +602,9 @@ def _bench_extra(args, sqa, torch, device, stream, flush, evict, peaks, lines):
                             for c in (0, 1):
                                 grid.append((N, H_q, H_kv, 128, c, 0.5, idx))
                             idx += 1
+            points = getattr(args, "sweep_points", None)
+            if points is not None:
+                grid = [g for g in grid if (g[0], g[1], g[2], g[4]) in points]
         for N, H_q, H_kv, d, causal, factor, seed in grid:
             _, dev = make_attn_inputs(1, N, H_q, H_kv, d, seed, factor, device)
             out = torch.empty((1, N, H_q, d), dtype=torch.bfloat16, device=device)
