@@ -63,7 +63,8 @@ def test_forward_odd_shapes(dbg, N, H_q, H_kv, causal):
 
 @pytest.mark.parametrize("B,N,H_q,H_kv,d,causal", [
     (2, 255, 4, 2, 128, False), (1, 1000, 8, 4, 128, True), (1, 640, 128, 1, 64, False),   # split: single tiles
-    (1, 4096, 4, 4, 64, False), (3, 300, 6, 4, 64, False)])                                 # split: pairs; uneven
+    (1, 4096, 4, 4, 64, False), (3, 300, 6, 4, 64, False),                                 # split: pairs; uneven
+    (1, 80, 8, 2, 128, True), (1, 161, 16, 1, 128, False), (1, 1600, 4, 4, 128, False)])  # d=128 80-key steps
 def test_forward_more_shapes(dbg, B, N, H_q, H_kv, d, causal):
     import torch
     qb, kb, vb = attn_inputs(B, N, H_q, H_kv, d, 42)

@@ -70,6 +70,27 @@ def test_edge_shapes_full_output(shape, causal):
     _full_check(*shape, causal, seed=11)
 
 
+# d=128 steps through the keys 80 at a time: lengths on and around those steps
+# (and shorter than one step), for every head stacking
+D128_STEPS = [
+    # B, N, H_q, H_kv, d
+    (1, 1, 2, 1, 128),
+    (1, 79, 4, 4, 128),
+    (1, 80, 8, 2, 128),
+    (1, 81, 16, 1, 128),
+    (2, 160, 4, 2, 128),
+    (1, 161, 8, 8, 128),
+    (1, 240, 32, 8, 128),
+    (1, 1600, 4, 4, 128),    # non-causal: a split last wave over an even number of key steps
+]
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("shape", D128_STEPS, ids=lambda s: "B%dN%dHq%dHkv%dd%d" % s)
+def test_d128_key_step_boundaries_full_output(shape, causal):
+    _full_check(*shape, causal, seed=12)
+
+
 @pytest.mark.parametrize("scale", [0.02, 0.3, 1.0])
 def test_nondefault_scale(scale):
     _full_check(1, 300, 4, 2, 64, True, scale=scale, seed=3)

@@ -37,6 +37,7 @@ CASES = [
     (1, 1000, 333, 200, 8, 4, 64),    # an interior block off the tile grid
     (2, 777, 700, 77, 16, 1, 64),     # the last rows, MQA with 16 heads stacked
     (1, 513, 1, 511, 12, 3, 128),     # all but the first row, d = 128
+    (1, 1000, 123, 300, 8, 2, 128),   # d = 128 block whose rows start off the 80-key step grid
     (3, 300, 150, 1, 6, 4, 64),       # one row, uneven groups
 ]
 
