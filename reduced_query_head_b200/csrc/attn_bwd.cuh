@@ -91,7 +91,8 @@ struct BwdParams {
 // core busy. dK/dV kernel at d = 64: K and V sit in TMEM, so all four products
 // are TS; warp 1 issues S^T and dV, warp 3 dP^T and dK, and every TMEM region
 // (scores or dP half of a buffer, one accumulator) has a single issuer. At
-// d = 128 there is no TMEM left for K and V; one issuer runs every product.
+// d = 128 there is no TMEM left for K and V: the score products read them from
+// shared memory (SS), with the same split of the products between the issuers.
 //   warp 0      TMA producer
 //   warp 1      MMA issuer 0 + TMEM owner
 //   warp 3      MMA issuer 1
@@ -121,9 +122,10 @@ template <int D>
 struct DkdvCfg {
   static constexpr int KCH = D / 64;                   // 128-byte column chunks
   static constexpr int BQ = 64;                        // queries per step
-  // d = 64: K and V rows in TMEM (A operands of the score products), two issuers
+  // d = 64: K and V rows in TMEM (A operands of the score products); d = 128:
+  // from shared memory. Two issuers either way, split by product.
   static constexpr bool KV_TMEM = (D == 64);
-  static constexpr int NI = KV_TMEM ? 2 : 1;
+  static constexpr int NI = 2;
   static constexpr int STAGES = (D == 64) ? 8 : 4;
   static constexpr int KV_BYTES = 128 * D * 2;         // K or V tile, 128 keys
   static constexpr int KV_CHUNK = 128 * 128;           // one column chunk of it
@@ -195,7 +197,7 @@ __global__ void __launch_bounds__(384, 1)
     for (int i = 0; i < C::N_BARS; ++i) {
       int cnt = 1;
       if (i == C::BAR_P || i == C::BAR_P + 1 || (C::KV_TMEM && i == C::BAR_KV)) cnt = 8;
-      else if (C::KV_TMEM && ((i >= C::BAR_S && i < C::BAR_S + 2) || (i >= C::BAR_EMPTY && i < C::BAR_EMPTY + C::STAGES))) cnt = 2;
+      else if (C::NI == 2 && ((i >= C::BAR_S && i < C::BAR_S + 2) || (i >= C::BAR_EMPTY && i < C::BAR_EMPTY + C::STAGES))) cnt = 2;
       mbar_init(bar(i), cnt);
     }
     *abort_flag = 0;
@@ -259,11 +261,12 @@ __global__ void __launch_bounds__(384, 1)
       const uint64_t dDm = sdesc_sw128(sbase + C::OFF_STAGE + C::T_BYTES, C::T_CHUNK, 1024);
       const uint32_t col_dv = tmem + C::COL_ACC, col_dk = col_dv + D;
       bool ok = mbar_wait(bar(C::BAR_KV), 0, ctl);
-      if (C::KV_TMEM) {
+      {
         // issuer 0: S^T = K Q_s^T into the buffer's first half, dV += P^T dO_s;
-        // issuer 1: dP^T = V dO_s^T into its second half, dK += dS^T Q_s
-        const uint32_t col_a = tmem + (me ? C::COL_VT : C::COL_KT);
+        // issuer 1: dP^T = V dO_s^T into its second half, dK += dS^T Q_s.
+        // Each TMEM region has one issuing thread, whose MMAs run in issue order.
         const uint64_t d_score = me ? dDk : dQk, d_grad = me ? dQm : dDm;
+        const uint64_t d_kv = me ? dV : dK;
         const uint32_t col_acc = me ? col_dk : col_dv, half = me ? 64u : 0u;
         auto issue_score = [&](int s) -> bool {
           const int st = s % C::STAGES;
@@ -271,9 +274,19 @@ __global__ void __launch_bounds__(384, 1)
           tc_fence_after();
           const uint64_t so = (uint64_t)(st * (C::STAGE_BYTES >> 4));
           const uint32_t buf = tmem + (uint32_t)(s & 1) * 128 + half;
+          if constexpr (C::KV_TMEM) {
+            const uint32_t col_a = tmem + (me ? C::COL_VT : C::COL_KT);
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk)
-            umma_ts(buf, col_a + kk * 8, d_score + so + (uint64_t)(((kk & 3) * 32) >> 4), IDESC_S, kk > 0);
+            for (int kk = 0; kk < D / 16; ++kk)
+              umma_ts(buf, col_a + kk * 8, d_score + so + (uint64_t)(((kk & 3) * 32) >> 4), IDESC_S, kk > 0);
+          } else {
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint64_t ok_ = ((kk >> 2) * C::KV_CHUNK + (kk & 3) * 32) >> 4;
+              const uint64_t oq = ((kk >> 2) * C::T_CHUNK + (kk & 3) * 32) >> 4;
+              umma_ss(buf, d_kv + ok_, d_score + so + oq, IDESC_S, kk > 0);
+            }
+          }
           umma_commit(bar(C::BAR_S + (s & 1)));
           return true;
         };
@@ -288,50 +301,12 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
           for (int kk = 0; kk < C::BQ / 16; ++kk)
             // queries 16kk.. were packed by warpgroup kk/2 into its 32 columns, chunk kk%2
+            // (B operands MN-major: d contiguous)
             umma_ts(col_acc, buf + (uint32_t)(32 * (kk >> 1) + 8 * (kk & 1)), d_grad + so + (uint64_t)((kk * 16 * 128) >> 4),
                     IDESC_G, (s > 0 || kk > 0) ? 1u : 0u);
           umma_commit(bar(C::BAR_EMPTY + st));
           // S^T / dP^T of step s + 2 overwrite what this issuer's own products just read
           if (s + 2 < n_steps) ok = issue_score(s + 2);
-        }
-      } else {
-        // S^T = K Q_s^T and dP^T = V dO_s^T into buffer s & 1
-        auto issue_scores = [&](int s) -> bool {
-          const int st = s % C::STAGES;
-          if (!mbar_wait(bar(C::BAR_FULL + st), (s / C::STAGES) & 1, ctl)) return false;
-          tc_fence_after();
-          const uint64_t so = (uint64_t)(st * (C::STAGE_BYTES >> 4));
-          const uint32_t buf = tmem + (uint32_t)(s & 1) * 128;
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint64_t ok_ = ((kk >> 2) * C::KV_CHUNK + (kk & 3) * 32) >> 4;
-            const uint64_t oq = ((kk >> 2) * C::T_CHUNK + (kk & 3) * 32) >> 4;
-            umma_ss(buf, dK + ok_, dQk + so + oq, IDESC_S, kk > 0);
-            umma_ss(buf + 64, dV + ok_, dDk + so + oq, IDESC_S, kk > 0);
-          }
-          umma_commit(bar(C::BAR_S + (s & 1)));
-          return true;
-        };
-        if (ok) ok = issue_scores(0);
-        if (ok && n_steps > 1) ok = issue_scores(1);
-        for (int s = 0; ok && s < n_steps; ++s) {
-          if (!mbar_wait_spin(bar(C::BAR_P + (s & 1)), (s >> 1) & 1, ctl)) { ok = false; break; }
-          tc_fence_after();
-          const int st = s % C::STAGES;
-          const uint64_t so = (uint64_t)(st * (C::STAGE_BYTES >> 4));
-          const uint32_t buf = tmem + (uint32_t)(s & 1) * 128;
-#pragma unroll
-          for (int kk = 0; kk < C::BQ / 16; ++kk) {
-            const uint32_t acc = (s > 0 || kk > 0) ? 1u : 0u;
-            const uint64_t ob = (uint64_t)((kk * 16 * 128) >> 4);
-            // dV += P^T dO_s and dK += dS^T Q_s (B operands MN-major: d contiguous)
-            // queries 16kk.. were packed by warpgroup kk/2 into its half, chunk kk%2
-            const uint32_t ca = (uint32_t)(32 * (kk >> 1) + 8 * (kk & 1));
-            umma_ts(col_dv, buf + ca, dDm + so + ob, IDESC_G, acc);
-            umma_ts(col_dk, buf + 64 + ca, dQm + so + ob, IDESC_G, acc);
-          }
-          umma_commit(bar(C::BAR_EMPTY + st));
-          if (s + 2 < n_steps) ok = issue_scores(s + 2);
         }
       }
       if (ok) umma_commit(bar(C::BAR_DONE + me));
