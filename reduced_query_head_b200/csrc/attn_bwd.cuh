@@ -79,16 +79,17 @@ struct BwdParams {
 
 
 
-// Both main kernels run a two-buffer pipeline over 64-column steps. TMEM
-// buffer b (b = step & 1) holds the step's scores in [128b, 128b + 64) and
-// its dP in [128b + 64, 128b + 128). Both elementwise warpgroups work on
-// every step, each on its own 32 of the 64 columns, and write P / dS back as
-// bf16 into the first 16 columns of their own 32 (the MMA reads each K16 step
-// of the A operand from wherever its warpgroup put it).
-// dQ kernel: each buffer has its own MMA issuer (warp 1 for even steps, warp 3
-// for odd steps) with its own dQ accumulator, summed in the epilogue: while one
-// issuer waits for the elementwise warps, the other's products keep the tensor
-// core busy. dK/dV kernel at d = 64: K and V sit in TMEM, so all four products
+// Both main kernels run a two-buffer pipeline: TMEM buffer b (b = step & 1)
+// holds the step's scores in its first half and dP in its second. Both
+// elementwise warpgroups work on every step, each on its own half of the
+// step's columns, and write P / dS back as bf16 behind the columns they have
+// already read (the MMA reads each K16 step of the A operand from wherever its
+// warpgroup put it). The MMA issuers are split by product, so every TMEM
+// region has one issuing thread and in-order issue orders its reuse.
+// dQ kernel (96-key steps, 192-column buffers): warp 1 issues S, warp 3 issues
+// dP and dQ += dS K_j into one dQ accumulator; Q and dO are TMEM operands at
+// d = 64 and shared-memory operands at d = 128.
+// dK/dV kernel (64-query steps): at d = 64 K and V sit in TMEM, so all four products
 // are TS; warp 1 issues S^T and dV, warp 3 dP^T and dK, and every TMEM region
 // (scores or dP half of a buffer, one accumulator) has a single issuer. At
 // d = 128 there is no TMEM left for K and V: the score products read them from
@@ -96,8 +97,8 @@ struct BwdParams {
 //   warp 0      TMA producer
 //   warp 1      MMA issuer 0 + TMEM owner
 //   warp 3      MMA issuer 1
-//   warps 4-7   elementwise, columns 0-31 of every step (thread = TMEM lane = tile row)
-//   warps 8-11  elementwise, columns 32-63 of every step
+//   warps 4-7   elementwise, first half of every step's columns (thread = TMEM lane = tile row)
+//   warps 8-11  elementwise, second half of every step's columns
 
 // 16 columns of the elementwise step from the scores s and dP read from TMEM:
 // p = exp2(s * scale_log2 - lse2), ds = p * (dP - D), both packed to bf16
@@ -434,19 +435,17 @@ __global__ void __launch_bounds__(384, 1)
 template <int D>
 struct DqCfg {
   static constexpr int KCH = D / 64;
-  // d = 64 (SPLIT): issuer 0 issues S, issuer 1 issues dP and dQ, so one dQ
-  // accumulator suffices and the TMEM it frees holds 96-key steps; d = 128:
-  // one issuer per buffer, each with its own dQ accumulator, 64-key steps.
-  static constexpr bool SPLIT = (D == 64);
-  static constexpr int BK = SPLIT ? 96 : 64;           // keys per step
-  static constexpr int STAGES = (D == 64) ? 8 : 4;
+  // Issuer 0 issues S, issuer 1 issues dP and dQ, so one dQ accumulator
+  // suffices and the TMEM it frees holds 96-key steps.
+  static constexpr int BK = 96;                        // keys per step
+  static constexpr int STAGES = (D == 64) ? 8 : 3;
   // d = 64: Q and dO live in TMEM as the A operands of the score products (TS
-  // form); at d = 128 the two issuers' accumulators fill TMEM and they stay in
-  // shared memory.
+  // form); at d = 128 the score buffers and the dQ accumulator fill TMEM and
+  // they stay in shared memory (SS form).
   static constexpr bool A_TMEM = (D == 64);
   static constexpr int Q_BYTES = 128 * D * 2;          // Q or dO tile, 128 rows
   static constexpr int Q_CHUNK = 128 * 128;
-  static constexpr int T_BYTES = BK * D * 2;           // K_j or V_j, 64 keys
+  static constexpr int T_BYTES = BK * D * 2;           // K_j or V_j, BK keys
   static constexpr int T_CHUNK = BK * 128;
   static constexpr int STAGE_BYTES = 2 * T_BYTES;
   static constexpr int OFF_Q = 0, OFF_DO = Q_BYTES, OFF_STAGE = A_TMEM ? 0 : 2 * Q_BYTES;
@@ -458,12 +457,10 @@ struct DqCfg {
   static constexpr int THREADS = 384;
   static constexpr uint32_t TMEM_COLS = 512;
   // TMEM buffer b at b * BUF: scores in [0, BK), dP in [BK, 2 BK). Then the dQ
-  // accumulator(s) (issuer i's at COL_DQ + i * D when not SPLIT), then the Q /
-  // dO rows (A_TMEM).
-  static constexpr uint32_t BUF = 2 * BK, N_ACC = SPLIT ? 1 : 2;
-  static constexpr uint32_t COL_DQ = 2 * BUF, COL_QT = COL_DQ + N_ACC * D, COL_DOT = COL_QT + D / 2;
-  static_assert(COL_DQ + N_ACC * D <= TMEM_COLS && (!A_TMEM || COL_DOT + D / 2 <= TMEM_COLS), "TMEM budget");
-  static_assert(!SPLIT || A_TMEM, "the split issuers take Q and dO from TMEM");
+  // accumulator, then the Q / dO rows (A_TMEM).
+  static constexpr uint32_t BUF = 2 * BK;
+  static constexpr uint32_t COL_DQ = 2 * BUF, COL_QT = COL_DQ + D, COL_DOT = COL_QT + D / 2;
+  static_assert(COL_DQ + D <= TMEM_COLS && (!A_TMEM || COL_DOT + D / 2 <= TMEM_COLS), "TMEM budget");
   // elementwise: each warpgroup owns CPW key columns of a step, in NCH chunks
   // of 16; chunk k of warpgroup w packs its dS into [w*CPW + 8k, +8) of the
   // buffer's dP half, behind the columns it has already read
@@ -515,11 +512,11 @@ __global__ void __launch_bounds__(384, 1)
 
   WaitCtl ctl{abort_flag, p.status, p.timeout_ns};
   if (tid == 0) {
-    // SPLIT: S and EMPTY take one commit from each issuer
+    // S and EMPTY take one commit from each issuer
     for (int i = 0; i < C::N_BARS; ++i) {
       int cnt = 1;
       if (i == C::BAR_P || i == C::BAR_P + 1 || (C::A_TMEM && i == C::BAR_QD)) cnt = 8;
-      else if (C::SPLIT && ((i >= C::BAR_S && i < C::BAR_S + 2) || (i >= C::BAR_EMPTY && i < C::BAR_EMPTY + C::STAGES)))
+      else if ((i >= C::BAR_S && i < C::BAR_S + 2) || (i >= C::BAR_EMPTY && i < C::BAR_EMPTY + C::STAGES))
         cnt = 2;
       mbar_init(bar(i), cnt);
     }
@@ -578,7 +575,7 @@ __global__ void __launch_bounds__(384, 1)
       const uint64_t dVk = sdesc_sw128(sbase + C::OFF_STAGE + C::T_BYTES, 16, 1024);
       const uint64_t dKm = sdesc_sw128(sbase + C::OFF_STAGE, C::T_CHUNK, 1024);
       bool ok = mbar_wait(bar(C::BAR_QD), 0, ctl);
-      if constexpr (C::SPLIT) {
+      {
         // issuer 0: S_j = Q K_j^T into the buffer's first half; issuer 1:
         // dP_j = dO V_j^T into its second half, then dQ += dS_j K_j with dS_j
         // read from that half. Each half has one issuing thread, so in-order
@@ -589,11 +586,21 @@ __global__ void __launch_bounds__(384, 1)
           tc_fence_after();
           const uint64_t so = (uint64_t)(st * (C::STAGE_BYTES >> 4));
           const uint32_t dst = tmem + (uint32_t)(j & 1) * C::BUF + (me ? (uint32_t)C::BK : 0u);
-          const uint32_t a_col = tmem + (me ? C::COL_DOT : C::COL_QT);
           const uint64_t b_desc = me ? dVk : dKk;
+          if constexpr (C::A_TMEM) {
+            const uint32_t a_col = tmem + (me ? C::COL_DOT : C::COL_QT);
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk)
-            umma_ts(dst, a_col + kk * 8, b_desc + so + (uint64_t)(((kk & 3) * 32) >> 4), IDESC_S, kk > 0);
+            for (int kk = 0; kk < D / 16; ++kk)
+              umma_ts(dst, a_col + kk * 8, b_desc + so + (uint64_t)(((kk & 3) * 32) >> 4), IDESC_S, kk > 0);
+          } else {
+            const uint64_t a_desc = me ? dO : dQ;
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint64_t oq = ((kk >> 2) * C::Q_CHUNK + (kk & 3) * 32) >> 4;
+              const uint64_t ok_ = ((kk >> 2) * C::T_CHUNK + (kk & 3) * 32) >> 4;
+              umma_ss(dst, a_desc + oq, b_desc + so + ok_, IDESC_S, kk > 0);
+            }
+          }
           umma_commit(bar(C::BAR_S + (j & 1)));
           return true;
         };
@@ -621,45 +628,6 @@ __global__ void __launch_bounds__(384, 1)
             umma_commit(bar(C::BAR_EMPTY + st));
             if (j + 2 < n_kv) ok = issue_score(j + 2);
           }
-        }
-      } else {
-        // S = Q K_j^T and dP = dO V_j^T into buffer j & 1
-        auto issue_scores = [&](int j) -> bool {
-          const int st = j % C::STAGES;
-          if (!mbar_wait(bar(C::BAR_FULL + st), (j / C::STAGES) & 1, ctl)) return false;
-          tc_fence_after();
-          const uint64_t so = (uint64_t)(st * (C::STAGE_BYTES >> 4));
-          const uint32_t buf = tmem + (uint32_t)(j & 1) * 128;
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint64_t ok_ = ((kk >> 2) * C::T_CHUNK + (kk & 3) * 32) >> 4;
-            if (C::A_TMEM) {
-              umma_ts(buf, tmem + C::COL_QT + kk * 8, dKk + so + ok_, IDESC_S, kk > 0);
-              umma_ts(buf + 64, tmem + C::COL_DOT + kk * 8, dVk + so + ok_, IDESC_S, kk > 0);
-            } else {
-              const uint64_t oq = ((kk >> 2) * C::Q_CHUNK + (kk & 3) * 32) >> 4;
-              umma_ss(buf, dQ + oq, dKk + so + ok_, IDESC_S, kk > 0);
-              umma_ss(buf + 64, dO + oq, dVk + so + ok_, IDESC_S, kk > 0);
-            }
-          }
-          umma_commit(bar(C::BAR_S + (j & 1)));
-          return true;
-        };
-        if (ok && me < n_kv) ok = issue_scores(me);
-        const uint32_t col_dq = tmem + C::COL_DQ + (uint32_t)me * D;
-        for (int j = me; ok && j < n_kv; j += 2) {
-          if (!mbar_wait_spin(bar(C::BAR_P + (j & 1)), (j >> 1) & 1, ctl)) { ok = false; break; }
-          tc_fence_after();
-          const int st = j % C::STAGES;
-          const uint64_t so = (uint64_t)(st * (C::STAGE_BYTES >> 4));
-          const uint32_t buf = tmem + (uint32_t)(j & 1) * 128;
-#pragma unroll
-          for (int kk = 0; kk < C::BK / 16; ++kk)
-            // dQ += dS K_j (K as an MN-major B operand: d contiguous)
-            umma_ts(col_dq, buf + (uint32_t)(32 * (kk >> 1) + 8 * (kk & 1)), dKm + so + (uint64_t)((kk * 16 * 128) >> 4), IDESC_G,
-                    (j > me || kk > 0) ? 1u : 0u);
-          umma_commit(bar(C::BAR_EMPTY + st));
-          if (j + 2 < n_kv) ok = issue_scores(j + 2);
         }
       }
       if (ok) umma_commit(bar(C::BAR_DONE + me));
@@ -735,7 +703,7 @@ __global__ void __launch_bounds__(384, 1)
         uint32_t pp[8], pd[8];
         bwd_chunk(ra, rb, sl2, nl, nd, pp, pd);
         // dS of chunk k into [8k, 8k + 8) of this warpgroup's dP columns (already read)
-        tmem_st8((C::SPLIT ? dpb : buf) + k * 8, pd);
+        tmem_st8(dpb + k * 8, pd);
         if (k + 1 < C::NCH) tmem_ld_wait16x2(ra2[(k + 1) & 1], rb2[(k + 1) & 1]);
       }
       tmem_st_wait();
@@ -743,28 +711,18 @@ __global__ void __launch_bounds__(384, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(C::BAR_P + (j & 1)));
     }
-    // epilogue: each warpgroup writes half of the row's d columns (x scale):
-    // the single accumulator of issuer 1 (SPLIT), else the sum of the two
-    // issuers' accumulators
-    const bool two = !C::SPLIT && n_kv > 1;
-    const bool acc_ready = ok && (C::SPLIT ? mbar_wait_warp(bar(C::BAR_DONE + 1), 0, ctl)
-                                           : (mbar_wait_warp(bar(C::BAR_DONE), 0, ctl) &&
-                                              (!two || mbar_wait_warp(bar(C::BAR_DONE + 1), 0, ctl))));
+    // epilogue: each warpgroup writes half of the row's d columns (x scale) of
+    // issuer 1's accumulator
+    const bool acc_ready = ok && mbar_wait_warp(bar(C::BAR_DONE + 1), 0, ctl);
     if (acc_ready) {
       tc_fence_after();
       const bool st = row_ok && in_bounds(head < p.H_q && b < p.B, p.status);
       __nv_bfloat16* dst = p.dq + (((size_t)b * p.N + (st ? token : 0)) * p.H_q + (st ? head : 0)) * D;
 #pragma unroll
       for (int c = wg * (D / 2); c < (wg + 1) * (D / 2); c += 32) {
-        uint32_t r[32], r1[32];
-        __syncwarp();   // after the per-lane stores: the TMEM loads are warp-collective
-        if (two) {
-          tmem_ld32x2(lane_base + C::COL_DQ + c, lane_base + C::COL_DQ + D + c, r, r1);
-#pragma unroll
-          for (int x = 0; x < 32; ++x) r[x] = __float_as_uint(__uint_as_float(r[x]) + __uint_as_float(r1[x]));
-        } else {
-          tmem_ld32(lane_base + C::COL_DQ + c, r);
-        }
+        uint32_t r[32];
+        __syncwarp();   // after the per-lane stores: the TMEM load is warp-collective
+        tmem_ld32(lane_base + C::COL_DQ + c, r);
         uint4 w[4];
         uint32_t* wp = reinterpret_cast<uint32_t*>(w);
 #pragma unroll
